@@ -1,0 +1,113 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every
+declared symbol, resolves pages on the host, and rejects bad arguments before
+touching CUDA (no compute call is made here)."""
+
+import ctypes
+import math
+import os
+
+import pytest
+
+from paged_kv_cache_exact_b200 import binding as B
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "worked_mapping.txt")
+
+
+def test_every_declared_symbol_is_exported():
+    names = B.declared_functions()
+    assert set(names) >= {"attn_prefill", "paged_attn", "paged_attn_workspace_size",
+                          "pkv_resolve", "pkv_last_device_error", "pkv_status_string"}
+    lib = ctypes.CDLL(B.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_resolve_matches_the_worked_example():
+    with open(GOLDEN) as f:
+        rows = [l.split() for l in f if l.strip() and not l.startswith("#")]
+    for kind, ps, table, token, *exp in rows:
+        if kind != "resolve":
+            continue
+        e = dict(x.split("=") for x in exp)
+        phys, off = B.pkv_resolve([int(x) for x in table.split(",")], int(ps), int(token))
+        assert (phys, off) == (int(e["physical"]), int(e["offset"]))
+
+
+def test_resolve_every_token_and_bounds():
+    table = [5, 1, 9]
+    for t in range(3 * 256):
+        assert B.pkv_resolve(table, 256, t) == (table[t // 256], t % 256)
+    with pytest.raises(B.PkvError) as ei:
+        B.pkv_resolve(table, 256, 3 * 256)
+    assert ei.value.status == B.PKV_ERR_INVALID_ARG
+
+
+def test_status_strings():
+    for s in range(7):
+        assert B.pkv_status_string(s) and B.pkv_status_string(s) != "unknown status"
+    assert B.pkv_status_string(99) == "unknown status"
+
+
+def test_workspace_size_plan():
+    # one split per sequence: no workspace
+    assert B.paged_attn_workspace_size(256, 32, 128, 200, 16) == 0
+    # the two decode workloads need one; the size covers (O, max, sum) per split
+    for S, L, ps in [(64, 8192, 16), (16, 32768, 256)]:
+        n = B.paged_attn_workspace_size(S, 32, 128, L, ps)
+        assert n > 0 and n >= S * 32 * 2 * (128 + 2) * 4
+        assert n == B.paged_attn_workspace_size(S, 32, 128, L, ps)   # deterministic
+    assert B.paged_attn_workspace_size(0, 32, 128, 8192, 16) == 0
+    assert B.paged_attn_workspace_size(4, 32, 128, 8192, 24) == 0
+
+
+FAKE = 1 << 20    # aligned non-null address; never dereferenced on these paths
+
+
+def _paged(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, table=FAKE, lens=FAKE, ps=16, S=2, q_len=1, H=4, H_kv=4,
+             d=128, P=8, maxp=4, max_len=64, causal=1, scale=0.1, dtype=B.PKV_BF16, out=FAKE,
+             ws=FAKE, ws_bytes=1 << 30, stream=None)
+    a.update(kw)
+    return B.raw_status("paged_attn", a["q"], a["k"], a["v"], a["table"], a["lens"], a["ps"],
+                        a["S"], a["q_len"], a["H"], a["H_kv"], a["d"], a["P"], a["maxp"],
+                        a["max_len"], a["causal"], ctypes.c_float(a["scale"]), a["dtype"],
+                        a["out"], a["ws"], ctypes.c_size_t(a["ws_bytes"]), a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), B.PKV_ERR_INVALID_ARG),
+    (dict(k=FAKE + 8), B.PKV_ERR_INVALID_ARG),            # misaligned
+    (dict(table=FAKE + 2), B.PKV_ERR_INVALID_ARG),
+    (dict(ps=8), B.PKV_ERR_INVALID_ARG),
+    (dict(ps=48), B.PKV_ERR_INVALID_ARG),
+    (dict(ps=512), B.PKV_ERR_INVALID_ARG),
+    (dict(H=6, H_kv=4), B.PKV_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), B.PKV_ERR_INVALID_ARG),
+    (dict(scale=0.0), B.PKV_ERR_INVALID_ARG),
+    (dict(causal=2), B.PKV_ERR_INVALID_ARG),
+    (dict(maxp=2, max_len=64), B.PKV_ERR_INVALID_ARG),    # table cannot hold max_len tokens
+    (dict(q_len=65), B.PKV_ERR_INVALID_ARG),              # max_len < q_len
+    (dict(d=96), B.PKV_ERR_UNSUPPORTED),
+    (dict(dtype=7), B.PKV_ERR_INVALID_ARG),
+    (dict(max_len=8192, maxp=512, ws=None, ws_bytes=0), B.PKV_ERR_WORKSPACE),
+    (dict(max_len=8192, maxp=512, ws_bytes=1024), B.PKV_ERR_WORKSPACE),
+    (dict(max_len=8192, maxp=512, ws=FAKE + 16), B.PKV_ERR_WORKSPACE),  # not 256-aligned
+])
+def test_paged_attn_rejects_bad_arguments(kw, status):
+    assert _paged(**kw) == status
+
+
+@pytest.mark.parametrize("args,status", [
+    ((None, FAKE, FAKE, FAKE, 1, 1, 16, 128, 1, 0.1, B.PKV_BF16), B.PKV_ERR_INVALID_ARG),
+    ((FAKE, FAKE, FAKE, FAKE + 4, 1, 1, 16, 128, 1, 0.1, B.PKV_BF16), B.PKV_ERR_INVALID_ARG),
+    ((FAKE, FAKE, FAKE, FAKE, 0, 1, 16, 128, 1, 0.1, B.PKV_BF16), B.PKV_ERR_INVALID_ARG),
+    ((FAKE, FAKE, FAKE, FAKE, 1, 1, 0, 128, 1, 0.1, B.PKV_BF16), B.PKV_ERR_INVALID_ARG),
+    ((FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 64, 1, 0.1, B.PKV_BF16), B.PKV_ERR_UNSUPPORTED),
+    ((FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 96, 1, 0.1, B.PKV_F32), B.PKV_ERR_UNSUPPORTED),
+    ((FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 128, 1, math.inf, B.PKV_BF16), B.PKV_ERR_INVALID_ARG),
+    ((FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 128, 1, 0.1, 5), B.PKV_ERR_INVALID_ARG),
+])
+def test_attn_prefill_rejects_bad_arguments(args, status):
+    *ptrs, Bn, H, N, d, causal, scale, dtype = args
+    assert B.raw_status("attn_prefill", *ptrs, Bn, H, N, d, causal, ctypes.c_float(scale),
+                        dtype, None) == status

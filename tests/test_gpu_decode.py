@@ -1,0 +1,134 @@
+"""Paged decode (q_len = 1, bf16) on the GPU against the fp64 oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from paged_kv_cache_exact_b200.workloads import make_paged, workload
+from tests._util import check_close, paged_ref_per_head, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(w, **kw):
+    from paged_kv_cache_exact_b200 import api
+    d = to_dev(w)
+    out = api.paged(d["q"], d["k"], d["v"], d["table"], d["lens"], w.page_size, w.causal,
+                    w.scale, max_seq_len=kw.get("max_seq_len", w.max_seq_len))
+    torch.cuda.synchronize()
+    return out.cpu()
+
+
+def _device_status():
+    from paged_kv_cache_exact_b200 import binding as B
+    return B.pkv_last_device_error()
+
+
+@pytest.mark.parametrize("ps", [16, 64, 256])
+@pytest.mark.parametrize("lens", [[1, 15, 16, 17], [300, 1000, 31, 4097], [2049]])
+def test_decode_small(ps, lens):
+    w = make_paged(11, lens, H=4, d=128, page_size=ps, q_len=1, decoys=3)
+    got = _run(w)
+    check_close(got, paged_ref_per_head(w), f"decode ps={ps} lens={lens}")
+    assert _device_status()[0] == 0
+
+
+def test_decode_gqa():
+    w = make_paged(12, [777, 64, 5000], H=32, H_kv=8, d=128, page_size=16, q_len=1)
+    check_close(_run(w), paged_ref_per_head(w), "decode gqa 32/8")
+
+
+def test_decode_aliased_pages():
+    """Two sequences share physical pages for a common prefix (pages 3 and 7,
+    as in the block-table example of "FlashAttention and PagedAttention: Two
+    Fixes for Two Different Bottlenecks"); pages are read-only, results exact."""
+    w = make_paged(13, [48, 48], H=2, d=128, page_size=16, q_len=1, decoys=0,
+                   fixed_tables={0: [3, 7, 12], 1: [3, 7, 9]}, pool_pages=13)
+    check_close(_run(w), paged_ref_per_head(w), "decode aliased")
+
+
+def test_decode_many_splits_and_max_len_slack():
+    # max_seq_len larger than any actual length: extra splits must be empty
+    w = make_paged(14, [5, 9000, 100], H=2, d=128, page_size=32, q_len=1)
+    pad = torch.full((3, 512 - w.block_table.shape[1]), -1, dtype=torch.int32)
+    w.block_table = torch.cat([w.block_table, pad], dim=1).contiguous()
+    check_close(_run(w, max_seq_len=16384), paged_ref_per_head(w), "decode slack")
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("cfg", [3, 4])
+def test_decode_full_workloads(cfg):
+    w = workload(cfg)
+    got = _run(w)
+    err, rel = check_close(got, paged_ref_per_head(w), f"workload {cfg}")
+    assert _device_status()[0] == 0
+    print(f"workload {cfg}: max abs err {err:.3e}, max rel err {rel:.3e}")
+
+
+def _sentinel_case(ps, lens, H, seed):
+    """Pages where each (seq, head) has one key that dominates by > 200 in the
+    exponent; its V row encodes (physical page, offset, seq, head) as small
+    integers exact in bf16, so the output must equal that row bit for bit."""
+    w = make_paged(seed, lens, H=H, d=128, page_size=ps, q_len=1, decoys=2)
+    table = w.block_table.numpy()
+    w.q[:] = 1.0
+    w.scale = 1.0
+    used = sorted(set(table[table >= 0].tolist()))
+    for p in used:                     # clear used pages (tails stay poisoned)
+        w.k_pages[p] = torch.where(torch.isnan(w.k_pages[p].float()), w.k_pages[p],
+                                   torch.zeros_like(w.k_pages[p]))
+        w.v_pages[p] = torch.where(torch.isnan(w.v_pages[p].float()), w.v_pages[p],
+                                   torch.zeros_like(w.v_pages[p]))
+    expect = np.zeros((len(lens), H, 1, 128))
+    rng = np.random.default_rng(seed)
+    for s, L in enumerate(lens):
+        for h in range(H):
+            # sweep page boundaries: first/last token of a page, and random ones
+            cands = [0, L - 1, min(L - 1, ps - 1), min(L - 1, ps), int(rng.integers(L))]
+            t = cands[(s * H + h) % len(cands)]
+            phys, off = oracle.resolve(table[s], ps, t)
+            w.k_pages[phys, off, h] = 2.0          # score 256 vs 0 elsewhere
+            code = [phys % 16, (phys // 16) % 16, (phys // 256) % 16, phys // 4096,
+                    off, s, h]
+            w.v_pages[phys, off, h, :7] = torch.tensor(code, dtype=torch.float32).to(w.v_pages.dtype)
+            expect[s, h, 0, :7] = code
+    return w, expect
+
+
+@pytest.mark.parametrize("ps,lens", [(256, [600, 300, 1]), (16, [33, 1024, 17, 999])])
+def test_sentinel_address_probe_bit_exact(ps, lens):
+    w, expect = _sentinel_case(ps, lens, H=4, seed=15)
+    got = _run(w).double().numpy()
+    assert np.array_equal(got, expect)
+
+
+def test_sentinel_worked_example_token_300():
+    """Token 300 of the 600-token sequence on pages [5, 1, 9] is read from
+    physical page 1, offset 44 (printed example), through the kernel."""
+    w = make_paged(16, [600], H=1, d=128, page_size=256, q_len=1, decoys=2,
+                   fixed_tables={0: [5, 1, 9]})
+    w.q[:] = 1.0
+    w.scale = 1.0
+    for p in (5, 1, 9):
+        w.k_pages[p] = torch.where(torch.isnan(w.k_pages[p].float()), w.k_pages[p],
+                                   torch.zeros_like(w.k_pages[p]))
+        w.v_pages[p] = torch.where(torch.isnan(w.v_pages[p].float()), w.v_pages[p],
+                                   torch.zeros_like(w.v_pages[p]))
+    w.k_pages[1, 44, 0] = 2.0
+    w.v_pages[1, 44, 0, 0] = 1.0      # physical page
+    w.v_pages[1, 44, 0, 1] = 44.0     # offset
+    got = _run(w)[0, 0, 0, :2].double().tolist()
+    assert got == [1.0, 44.0]
+
+
+def test_bad_page_id_is_flagged_not_faulted():
+    from paged_kv_cache_exact_b200 import binding as B
+    w = make_paged(17, [64, 64], H=2, d=128, page_size=16, q_len=1)
+    w.block_table[1, 2] = w.k_pages.shape[0] + 5          # out of range for seq 1
+    _device_status()                                       # clear
+    got = _run(w)
+    st, bits = _device_status()
+    assert st == B.PKV_ERR_BAD_TABLE and bits & B.PKV_DEVERR_BAD_PAGE
+    # sequence 0 is untouched by the bad entry
+    check_close(got[:1], paged_ref_per_head(w, seqs=[0]), "good sequence")
