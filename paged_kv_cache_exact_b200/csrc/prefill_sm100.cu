@@ -1,5 +1,532 @@
-// placeholder, replaced by the tcgen05 prefill kernel
+// Tensor-core attention prefill for sm_100a (bf16 in/out, f32 accumulation).
+//
+// The method is the tiled online softmax of "Flash Attention: Fast,
+// Memory-Efficient Attention for LLMs", section "The Algorithm": for each K/V
+// tile, S = Q K^T, a running row max m and row sum l, P = exp(S - m), and the
+// output accumulator rescaled when m moves; S and P never leave the SM.  Its
+// "Flash Attention 2" section's causal skip is kept (tiles past the diagonal
+// are never loaded).  K/V come either from contiguous [B, H_kv, N, d] tensors
+// or, for paged prefill, straight from the pages through the block table
+// ("What is Paged FlashAttention?", "How does it work?"), one TMA box per page.
+//
+// The B200 design (the pages' H100/SRAM tiling is prior art only):
+//
+// * CTA = two 128-row Q tiles of one (batch, head) sharing every K/V tile.
+//   Warp roles: warps 0-3 and 4-7 are the softmax warpgroups of Q tile 0 and 1
+//   (one thread per row = one TMEM lane), warp 8 issues TMA loads, warp 9
+//   issues tcgen05.mma from one elected lane.
+// * TMEM (512 columns x 128 lanes x 32 bit): S0 | S1 | O0 | O1, 128 f32 columns
+//   each.  P (bf16) overwrites the first 64 columns of its S once the softmax
+//   has read S into registers, and feeds the PV product straight from TMEM
+//   (A operand in tensor memory), so P never touches shared memory.
+// * Shared memory: Q0, Q1 and a 2-stage ring for K and one for V, 32 KB per
+//   128x128 bf16 tile, all in the 128-byte-swizzled K-major layout TMA writes.
+// * Issue order on the MMA warp is S0(j+1) right after PV0(j) and S1(j+1)
+//   right after PV1(j): while the softmax of one Q tile runs, the tensor core
+//   works on the other tile (ping-pong).  tcgen05.mma executes in issue order,
+//   so S_i(j+1) may overwrite P_i(j) once PV_i(j) has been issued.
+// * Online softmax in base 2 with the scale folded into one FFMA; the output
+//   is rescaled only when the running max grows by more than 2^8 (exact: O and
+//   l always share the same reference max, and p stays <= 2^8).
+// * Every mbarrier wait is bounded (about 2 s); on expiry the CTA records
+//   PKV_DEVERR_TIMEOUT, stops issuing work, drains what it already issued and
+//   frees its TMEM.
+#include <cuda.h>
+
+#include <mutex>
+
 #include "common.cuh"
+#include "sm100_ptx.cuh"
+
 namespace pkv {
-cudaError_t launch_prefill_bf16(const PrefillParams&, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+using namespace sm100;
+
+constexpr int D = 128;             // head dim
+constexpr int BM = 128;            // rows per Q tile
+constexpr int BN = 128;            // keys per K/V tile
+constexpr int kQTiles = 2;         // Q tiles per CTA
+constexpr int kStages = 2;         // K ring and V ring depth
+constexpr int kThreads = 320;      // 10 warps
+constexpr int kTileBytes = BM * D * 2;             // 32 KB
+constexpr int kHalfBytes = kTileBytes / 2;         // one 64-column block: 16 KB
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
+constexpr float kRescaleThreshold = 8.0f;          // log2 units
+
+// Shared memory map (offsets from a 1024-aligned base).
+constexpr int kOffQ = 0;
+constexpr int kOffK = kOffQ + kQTiles * kTileBytes;
+constexpr int kOffV = kOffK + kStages * kTileBytes;
+constexpr int kOffBar = kOffV + kStages * kTileBytes;
+enum Bar {
+  kBarQ = 0,
+  kBarKFull = 1,                      // + stage
+  kBarKEmpty = kBarKFull + kStages,   // + stage
+  kBarVFull = kBarKEmpty + kStages,
+  kBarVEmpty = kBarVFull + kStages,
+  kBarSFull = kBarVEmpty + kStages,   // + q tile
+  kBarPFull = kBarSFull + kQTiles,
+  kBarODone = kBarPFull + kQTiles,
+  kBarVFixed = kBarODone + kQTiles,   // last paged V tile after tail rows are zeroed
+  kBarDrain = kBarVFixed + 1,
+  kNumBars = kBarDrain + 1
+};
+constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
+constexpr int kOffAbort = kOffTmemSlot + 4;
+constexpr int kSmemUsed = kOffAbort + 4;
+constexpr int kSmemBytes = kSmemUsed + 1024;       // slack for 1024-byte alignment
+
+// TMEM columns.
+constexpr uint32_t kColS = 0;      // + 128 * tile
+constexpr uint32_t kColO = 256;    // + 128 * tile
+
+constexpr uint32_t kIdescS = make_idesc_bf16(BM, BN, false);  // Q (K-major) x K (K-major)
+constexpr uint32_t kIdescO = make_idesc_bf16(BM, D, true);    // P (TMEM) x V (MN-major)
+
+struct Geometry {
+  int b, h, kvh, q0, q_len, kv_len, off, n_tiles;
+};
+
+__device__ __forceinline__ Geometry cta_geometry(const PrefillParams& p) {
+  Geometry g;
+  const int bh = blockIdx.x;
+  g.b = bh / p.H;
+  g.h = bh % p.H;
+  g.kvh = g.h / (p.H / p.H_kv);
+  g.q0 = (gridDim.y - 1 - blockIdx.y) * (BM * kQTiles);   // heaviest causal blocks first
+  g.q_len = p.q_len;
+  int kv_len = p.kv_len;
+  if (p.paged) {
+    kv_len = p.seq_lens[g.b];
+    const int cap = min(p.max_seq_len, p.max_pages * p.page_size);
+    if (kv_len < p.q_len || kv_len > cap) {
+      if (blockIdx.y == 0 && g.h == 0 && threadIdx.x == 0) flag_error(p.err, PKV_DEVERR_BAD_LEN);
+      kv_len = max(0, min(kv_len, cap));
+    }
+  }
+  g.kv_len = kv_len;
+  g.off = kv_len - p.q_len;
+  int n = (kv_len + BN - 1) / BN;
+  if (p.causal) {
+    const int last_row = min(g.q0 + BM * kQTiles - 1, p.q_len - 1);
+    const int last_key = last_row + g.off;      // may be < 0: nothing visible
+    n = last_key < 0 ? 0 : min(n, last_key / BN + 1);
+  }
+  g.n_tiles = max(n, 0);
+  return g;
 }
+
+// ----------------------------------------------------------------------------
+template <bool kPaged>
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto bar = [&](int i) { return sbase + kOffBar + 8 * i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const Geometry g = cta_geometry(p);
+  const int n = g.n_tiles;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kNumBars; ++i) {
+      const uint32_t cnt = (i == kBarPFull || i == kBarPFull + 1) ? 128u : 1u;
+      mbar_init(bar(i), cnt);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(sbase + kOffTmemSlot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kOffTmemSlot);
+
+  auto fail = [&]() {
+    *abort_flag = 1;
+    flag_error(p.err, PKV_DEVERR_TIMEOUT);
+  };
+  auto wait = [&](int b, uint32_t parity) -> bool {
+    if (*abort_flag) return false;
+    if (!mbar_wait_bounded(bar(b), parity, kWaitLimitNs)) {
+      fail();
+      return false;
+    }
+    return true;
+  };
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0 && n > 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      const int qc2 = g.b * p.H + g.h;
+      mbar_arrive_expect_tx(bar(kBarQ), kQTiles * kTileBytes);
+      for (int t = 0; t < kQTiles; ++t)
+        for (int c = 0; c < 2; ++c)
+          tma_load_3d(sbase + kOffQ + t * kTileBytes + c * kHalfBytes, &tmQ, c * 64,
+                      g.q0 + t * BM, qc2, bar(kBarQ));
+      int last_k = -1, last_v = -1;                  // last tile whose K / V load was issued
+      const int rows_per_box = kPaged ? min(p.page_size, BN) : BN;
+      const int n_valid_pages = kPaged ? (g.kv_len + p.page_size - 1) >> p.page_shift : 0;
+      // Token row of box i of tile j in the page pool (paged) -- ids outside
+      // the pool are flagged and replaced by page 0, so nothing outside it is read.
+      auto box_row = [&](int k0, int i) -> int {
+        const int t = k0 + i * rows_per_box;
+        int phys = p.block_table[(size_t)g.b * p.max_pages + (t >> p.page_shift)];
+        if (phys < 0 || phys >= p.num_pages) {
+          flag_error(p.err, PKV_DEVERR_BAD_PAGE);
+          phys = 0;
+        }
+        return phys * p.page_size + (t & (p.page_size - 1));
+      };
+      auto load_tile = [&](const CUtensorMap* tm, uint32_t smem_tile, uint32_t full_bar, int k0,
+                           int nbox) {
+        for (int c = 0; c < 2; ++c) {
+          const uint32_t dst = smem_tile + c * kHalfBytes;
+          if (kPaged) {
+            for (int i = 0; i < nbox; ++i)
+              tma_load_3d(dst + i * rows_per_box * 128, tm, c * 64, g.kvh, box_row(k0, i), full_bar);
+          } else {
+            tma_load_3d(dst, tm, c * 64, k0, g.b * p.H_kv + g.kvh, full_bar);
+          }
+        }
+      };
+      bool ok = true;
+      for (int j = 0; j < n && ok; ++j) {
+        const int st = j % kStages;
+        const uint32_t ph = (j / kStages) & 1;
+        const int k0 = j * BN;
+        // boxes of this tile that hold tokens of the sequence (never past its last page)
+        const int nbox = kPaged ? min(BN / rows_per_box, n_valid_pages - (k0 >> p.page_shift)) : 1;
+        const uint32_t bytes = kPaged ? nbox * rows_per_box * 256 : kTileBytes;
+        ok = wait(kBarKEmpty + st, ph ^ 1);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar(kBarKFull + st), bytes);
+        load_tile(&tmK, sbase + kOffK + st * kTileBytes, bar(kBarKFull + st), k0, nbox);
+        last_k = j;
+        ok = wait(kBarVEmpty + st, ph ^ 1);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar(kBarVFull + st), bytes);
+        load_tile(&tmV, sbase + kOffV + st * kTileBytes, bar(kBarVFull + st), k0, nbox);
+        last_v = j;
+      }
+      if (!ok) {
+        // Drain loads already in flight before the CTA's shared memory goes away.
+        for (int jj = max(0, last_k - 1); jj <= last_k; ++jj)
+          mbar_wait_bounded(bar(kBarKFull + jj % kStages), (jj / kStages) & 1, kWaitLimitNs);
+        for (int jj = max(0, last_v - 1); jj <= last_v; ++jj)
+          mbar_wait_bounded(bar(kBarVFull + jj % kStages), (jj / kStages) & 1, kWaitLimitNs);
+      }
+    }
+    // Paged, last tile partial: rows past kv_len (poisoned tails, unread pages)
+    // must be zero in V, since P = 0 there but 0 * NaN is NaN.  The whole warp
+    // zeroes them once the tile has landed, then releases it to the MMA warp.
+    if (kPaged && n > 0) {
+      const int j = n - 1;
+      const int valid = g.kv_len - j * BN;
+      if (valid < BN) {
+        __syncwarp();
+        const int st = j % kStages;
+        bool ok = !*abort_flag;
+        if (lane == 0 && ok) ok = mbar_wait_bounded(bar(kBarVFull + st), (j / kStages) & 1, kWaitLimitNs);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (ok) {
+          uint8_t* vt = smem + kOffV + st * kTileBytes;
+          const int nrows = BN - valid;
+          for (int idx = lane; idx < nrows * 16; idx += 32) {       // 16 x 16 B per row (2 blocks)
+            const int r = valid + idx / 16, part = idx % 16;
+            *reinterpret_cast<uint4*>(vt + (part / 8) * kHalfBytes + r * 128 + (part % 8) * 16) =
+                make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(kBarVFixed));
+        } else if (lane == 0) {
+          fail();
+        }
+      }
+    }
+  } else if (warp == 9) {
+    // ----------------------------------------------------------------- MMA --
+    if (lane == 0 && n > 0) {
+      const uint32_t sQ = sbase + kOffQ;
+      const bool last_fix = kPaged && (g.kv_len - (n - 1) * BN) < BN;
+      auto issue_s = [&](int t, int j) {
+        const int st = j % kStages;
+        const uint32_t sK = sbase + kOffK + st * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk / 4) * kHalfBytes + (kk % 4) * 32;
+          const uint64_t da = make_sdesc(sQ + t * kTileBytes + koff, 16, 1024);
+          const uint64_t db = make_sdesc(sK + koff, 16, 1024);
+          mma_ss(tmem + kColS + 128 * t, da, db, kIdescS, kk > 0);
+        }
+        mma_commit(bar(kBarSFull + t));
+      };
+      auto issue_pv = [&](int t, int j) {
+        const int st = j % kStages;
+        const uint32_t sV = sbase + kOffV + st * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t db = make_sdesc(sV + kk * 16 * 128, kHalfBytes, 1024);
+          mma_ts(tmem + kColO + 128 * t, tmem + kColS + 128 * t + kk * 8, db, kIdescO,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(bar(kBarODone + t));
+      };
+      bool ok = wait(kBarQ, 0) && wait(kBarKFull + 0, 0);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+        mma_commit(bar(kBarKEmpty + 0));
+      }
+      for (int j = 0; j < n && ok; ++j) {
+        const int st = j % kStages;
+        const uint32_t ph = (j / kStages) & 1;
+        if (last_fix && j == n - 1)
+          ok = wait(kBarVFixed, 0);
+        else
+          ok = wait(kBarVFull + st, ph);
+        ok = ok && wait(kBarPFull + 0, j & 1);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(0, j);
+        if (j + 1 < n) {
+          const int st1 = (j + 1) % kStages;
+          ok = wait(kBarKFull + st1, ((j + 1) / kStages) & 1);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(0, j + 1);
+        }
+        ok = wait(kBarPFull + 1, j & 1);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(1, j);
+        mma_commit(bar(kBarVEmpty + st));
+        if (j + 1 < n) {
+          issue_s(1, j + 1);
+          mma_commit(bar(kBarKEmpty + (j + 1) % kStages));
+        }
+      }
+      if (!ok) {
+        // Let every MMA already issued finish before TMEM is released.
+        mma_commit(bar(kBarDrain));
+        mbar_wait_bounded(bar(kBarDrain), 0, kWaitLimitNs);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------- softmax --
+    const int t = warp >> 2;                         // Q tile of this warpgroup
+    const int r = threadIdx.x & 127;                 // row in tile = TMEM lane
+    const int row = g.q0 + t * BM + r;               // query row
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_addr + kColS + 128 * t;
+    const uint32_t tO = tmem + lane_addr + kColO + 128 * t;
+    const float c = p.scale_log2;
+    const int limit = p.causal ? min(row + g.off, g.kv_len - 1) : g.kv_len - 1;
+
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    // tcgen05.ld/st are warp-collective: every branch around them is warp-uniform.
+    for (int j = 0; j < n; ++j) {
+      ok = wait(kBarSFull + t, j & 1);
+      if (ok && j > 0) ok = wait(kBarODone + t, (j - 1) & 1);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t s[128];
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t (&sub)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[32 * ch]);
+        tmem_ld32(tS + 32 * ch, sub);
+      }
+      tmem_wait_ld();
+      const int k0 = j * BN;
+      float mx = -INFINITY;
+      if (k0 + BN - 1 > limit) {                     // diagonal or tail tile: mask
+#pragma unroll
+        for (int i = 0; i < 128; ++i) {
+          const float v = (k0 + i <= limit) ? __uint_as_float(s[i]) : -INFINITY;
+          s[i] = __float_as_uint(v);
+          mx = fmaxf(mx, v);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 128; ++i) mx = fmaxf(mx, __uint_as_float(s[i]));
+      }
+      const float m_tile = mx * c;                  // running max in log2 units
+      float alpha = 1.f;
+      bool rescale = false;
+      if (m_tile > m_ref + kRescaleThreshold || (m_ref == -INFINITY && m_tile != -INFINITY)) {
+        alpha = ex2(m_ref - m_tile);               // m_ref = -inf -> 0
+        m_ref = m_tile;
+        rescale = true;
+      }
+      const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+      float rowsum = 0.f;
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {            // 64 scores -> 32 packed bf16 pairs
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float p0 = ex2(fmaf(__uint_as_float(s[64 * ch + 2 * i]), c, neg_m));
+          const float p1 = ex2(fmaf(__uint_as_float(s[64 * ch + 2 * i + 1]), c, neg_m));
+          rowsum += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(tS + 32 * ch, pk);
+      }
+      if (__any_sync(0xffffffffu, rescale) && j > 0) {   // alpha = 1 in rows that keep m
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * ch, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tO + 32 * ch, o);
+        }
+      }
+      l = l * alpha + rowsum;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(kBarPFull + t));
+    }
+    if (ok && n > 0) ok = wait(kBarODone + t, (n - 1) & 1);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) tc_fence_after();
+    // Epilogue: O / l -> bf16 -> global (rows past q_len are not stored).
+    const bool have_o = ok && n > 0;                 // warp-uniform
+    const bool store = row < g.q_len;
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.O) +
+                         (((size_t)g.b * p.H + g.h) * p.q_len + (store ? row : 0)) * D;
+    const float inv = (have_o && l > 0.f) ? 1.f / l : 0.f;
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
+      uint32_t o[32];
+      if (have_o) {
+        tmem_ld32(tO + 32 * ch, o);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = 0u;
+      }
+      if (store) {
+        uint4 packed[4];
+        uint32_t* pw = reinterpret_cast<uint32_t*>(packed);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pw[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+        uint4* dst = reinterpret_cast<uint4*>(out + 32 * ch);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dst[i] = packed[i];
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ----------------------------------------------------------------- host side --
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                              const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                              const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn get_encode() {
+  static EncodeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(ptr);
+  });
+  return fn;
+}
+
+// 3-D bf16 map, 128-byte swizzle, box {64, box1, box2}; out-of-range reads fill zeros.
+bool encode_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+               uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box1, uint32_t box2) {
+  EncodeFn enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+  const cuuint32_t box[3] = {64, box1, box2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+template <bool kPaged>
+cudaError_t set_smem_attr() {
+  static int done[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<kPaged>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = 1;
+  return e;
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_bf16(const PrefillParams& p, cudaStream_t stream) {
+  if (p.d != D) return cudaErrorNotSupported;
+  CUtensorMap tq, tk, tv;
+  const uint64_t row_bytes = D * 2;
+  // Q: [B*H, q_len, d]
+  if (!encode_3d(&tq, p.Q, D, p.q_len, (uint64_t)p.B * p.H, row_bytes, row_bytes * p.q_len, BM, 1))
+    return cudaErrorInvalidValue;
+  if (p.paged) {
+    // pages [P, ps, H_kv, d] viewed as [P*ps tokens, H_kv, d]; one box = one page's rows.
+    const uint32_t rows = p.page_size < BN ? p.page_size : BN;
+    const uint64_t tokens = (uint64_t)p.num_pages * p.page_size;
+    if (!encode_3d(&tk, p.K, D, p.H_kv, tokens, row_bytes, row_bytes * p.H_kv, 1, rows) ||
+        !encode_3d(&tv, p.V, D, p.H_kv, tokens, row_bytes, row_bytes * p.H_kv, 1, rows))
+      return cudaErrorInvalidValue;
+  } else {
+    const uint64_t bhkv = (uint64_t)p.B * p.H_kv;
+    if (!encode_3d(&tk, p.K, D, p.kv_len, bhkv, row_bytes, row_bytes * p.kv_len, BN, 1) ||
+        !encode_3d(&tv, p.V, D, p.kv_len, bhkv, row_bytes, row_bytes * p.kv_len, BN, 1))
+      return cudaErrorInvalidValue;
+  }
+  const int m_blocks = (p.q_len + BM * kQTiles - 1) / (BM * kQTiles);
+  if (m_blocks > 65535) return cudaErrorNotSupported;
+  dim3 grid((unsigned)p.B * p.H, m_blocks);
+  cudaError_t e;
+  if (p.paged) {
+    e = set_smem_attr<true>();
+    if (e != cudaSuccess) return e;
+    prefill_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, p);
+  } else {
+    e = set_smem_attr<false>();
+    if (e != cudaSuccess) return e;
+    prefill_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, p);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace pkv

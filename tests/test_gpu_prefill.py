@@ -1,0 +1,134 @@
+"""Tensor-core prefill (bf16) on the GPU against the fp64 oracle: contiguous and
+paged K/V, causal and not, ragged sizes, chunked (q_len < kv_len), GQA, and the
+full-size workloads on sampled rows."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from paged_kv_cache_exact_b200.workloads import make_dense, make_paged, workload
+from tests._util import check_close, f64, np_of, paged_ref_per_head, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _status_ok():
+    from paged_kv_cache_exact_b200 import binding as B
+    st, bits = B.pkv_last_device_error()
+    assert st == 0, f"device error word {bits:#x}"
+
+
+def _dense(w):
+    from paged_kv_cache_exact_b200 import api
+    out = api.prefill(w.Q.cuda(), w.K.cuda(), w.V.cuda(), w.causal, w.scale)
+    torch.cuda.synchronize()
+    return out.cpu()
+
+
+def _paged(w, max_seq_len=None):
+    from paged_kv_cache_exact_b200 import api
+    d = to_dev(w)
+    out = api.paged(d["q"], d["k"], d["v"], d["table"], d["lens"], w.page_size, w.causal,
+                    w.scale, max_seq_len=max_seq_len or w.max_seq_len)
+    torch.cuda.synchronize()
+    return out.cpu()
+
+
+@pytest.mark.parametrize("N", [1, 5, 127, 128, 129, 255, 256, 257, 300, 513, 1000])
+@pytest.mark.parametrize("causal", [True, False])
+def test_dense_small(N, causal):
+    w = make_dense(31 + N, 1, 2, N, 128, causal=causal)
+    got = _dense(w)
+    want = oracle.mha_ref(f64(w.Q), f64(w.K), f64(w.V), causal, w.scale)
+    check_close(got, want, f"dense N={N} causal={causal}")
+    _status_ok()
+
+
+def test_dense_batch_heads_and_scale():
+    w = make_dense(41, 3, 5, 700, 128, causal=True, scale=0.05)
+    got = _dense(w)
+    want = oracle.mha_ref(f64(w.Q), f64(w.K), f64(w.V), True, 0.05)
+    check_close(got, want, "dense B=3 H=5")
+    _status_ok()
+
+
+def test_dense_large_scores_no_overflow():
+    # scores far above exp's fp32 range: the running max keeps every exp <= 2^8
+    w = make_dense(42, 1, 2, 384, 128, causal=True, scale=2.0)
+    got = _dense(w)
+    want = oracle.mha_ref(f64(w.Q), f64(w.K), f64(w.V), True, 2.0)
+    check_close(got, want, "dense large scores")
+
+
+@pytest.mark.slow
+def test_causal_prefill_workload_sampled_rows():
+    """4 x 32 x 4096 x 128 causal: every head on 40 rows spanning tile edges,
+    and two heads in full."""
+    w = workload(2)
+    got = _dense(w)
+    rows = np.array(sorted({0, 1, 127, 128, 129, 255, 256, 511, 1023, 2047, 2048, 4094, 4095} |
+                           set(np.random.default_rng(2).integers(0, 4096, 27).tolist())))
+    Q, K, V = np_of(w.Q), np_of(w.K), np_of(w.V)
+    for b in range(4):
+        want = oracle.mha_ref(Q[b:b + 1], K[b:b + 1], V[b:b + 1], True, w.scale, rows=rows)
+        check_close(got[b:b + 1, :, rows], want, f"workload 2 batch {b}")
+    for b, h in [(0, 0), (3, 31)]:
+        want = oracle.attention_ref(Q[b, h], K[b, h], V[b, h], True, w.scale)
+        check_close(got[b, h], want, f"workload 2 head ({b},{h})")
+    _status_ok()
+
+
+@pytest.mark.parametrize("ps", [16, 64, 128, 256])
+@pytest.mark.parametrize("lens", [[200, 1000], [128, 513, 37]])
+def test_paged_full_prefill(ps, lens):
+    # q_len = min(lens) so every sequence has q_len <= kv_len (chunked for the longer ones)
+    q_len = min(lens)
+    w = make_paged(51 + ps, lens, H=2, d=128, page_size=ps, q_len=q_len, decoys=3)
+    got = _paged(w)
+    check_close(got, paged_ref_per_head(w), f"paged ps={ps} lens={lens}")
+    _status_ok()
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_paged_chunked_prefill_gqa(causal):
+    w = make_paged(61, [300, 700, 1025], H=8, H_kv=2, d=128, page_size=32, q_len=300,
+                   causal=causal)
+    got = _paged(w)
+    check_close(got, paged_ref_per_head(w), f"paged chunked gqa causal={causal}")
+    _status_ok()
+
+
+def test_paged_equals_contiguous_bit_identical():
+    """The same K/V as a contiguous tensor, as pages in order, and as shuffled
+    pages: the three results are bit-identical (same tiles, same order)."""
+    from paged_kv_cache_exact_b200 import api
+    N, H, ps = 640, 2, 64
+    w = make_dense(71, 1, H, N, 128, causal=True)
+    dense = _dense(w)
+    n_pages = N // ps
+    for perm in (np.arange(n_pages), np.random.default_rng(7).permutation(n_pages)):
+        k_pages = torch.empty(n_pages + 2, ps, H, 128, dtype=torch.bfloat16).fill_(float("nan"))
+        v_pages = k_pages.clone()
+        for lp in range(n_pages):
+            k_pages[perm[lp]] = w.K[0, :, lp * ps:(lp + 1) * ps].transpose(0, 1)
+            v_pages[perm[lp]] = w.V[0, :, lp * ps:(lp + 1) * ps].transpose(0, 1)
+        table = torch.tensor(perm, dtype=torch.int32)[None]
+        out = api.paged(w.Q.cuda(), k_pages.cuda(), v_pages.cuda(), table.cuda(),
+                        torch.tensor([N], dtype=torch.int32).cuda(), ps, True, w.scale,
+                        max_seq_len=N).cpu()
+        assert torch.equal(out.view(torch.int16), dense.view(torch.int16))
+
+
+@pytest.mark.slow
+def test_long_paged_prefill_workload_sampled_rows():
+    """1 x 32 x 32768 x 128 causal from 128 shuffled pages of 256: every head on
+    256 rows including the tile and page edges."""
+    w = workload(5)
+    got = _paged(w)
+    rng = np.random.default_rng(5)
+    fixed = [0, 1, 127, 128, 255, 256, 257, 16383, 32766, 32767]
+    rows = np.array(sorted(set(fixed) | set(rng.integers(0, 32768, 246).tolist())))
+    want = paged_ref_per_head(w, rows=rows)
+    check_close(got[:, :, rows], want, "workload 5")
+    _status_ok()
