@@ -149,6 +149,41 @@ PKV_API int paged_attn(const void* q, const void* k_pages, const void* v_pages,
                void* out, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * paged_decode_noalloc - paged decode that allocates nothing and needs no
+ * workspace argument.
+ *
+ * The pages have no counterpart for this entry point; it exists for callers
+ * that cannot allocate device memory where they call attention: a plugin
+ * invoked from another runtime's enqueue hook that offers no allocator, a
+ * latency-critical loop in which cudaMalloc/cudaFree would synchronise the
+ * device, or a process whose device memory a pool has reserved in full.
+ *
+ * It computes what paged_attn computes for q_len == 1 and PKV_BF16 (decode:
+ * every cached key is visible), with the same kernels and split plan, and the
+ * same meaning, layout and validation of the arguments paged_attn shares with
+ * it (d must be 128).  The split partials live in a static device array of
+ * PKV_NOALLOC_SCRATCH_BYTES inside the library: every GPU that loads the
+ * library holds that memory until the process exits.
+ *
+ * - Limit: when paged_attn_workspace_size(num_seqs, H, d, max_seq_len,
+ *   page_size) exceeds PKV_NOALLOC_SCRATCH_BYTES the call returns
+ *   PKV_ERR_WORKSPACE and launches nothing.
+ * - Set-up: the first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *   first call before any stream capture.
+ * - Sharing: all calls on a device use the same array, which keeps the last
+ *   call's contents.  No part of it needs to start at zero (a call writes every
+ *   partial it reads), but calls whose kernels overlap on the GPU (other
+ *   streams, other host threads) race on it: serialise them.
+ */
+#define PKV_NOALLOC_SCRATCH_BYTES (64u << 20)
+PKV_API int paged_decode_noalloc(const void* q, const void* k_pages, const void* v_pages,
+                                 const int32_t* block_table, const int32_t* seq_lens,
+                                 int page_size, int num_seqs, int H, int H_kv, int d,
+                                 int num_pages, int max_pages_per_seq, int max_seq_len,
+                                 float scale, void* out, void* stream);
+
+/*
  * pkv_resolve - host-side page-table address resolution (for tests and tools).
  *
  * Defines: "What is Paged FlashAttention?", section "Practical example".

@@ -30,6 +30,7 @@ PKV_OK, PKV_ERR_INVALID_ARG, PKV_ERR_UNSUPPORTED, PKV_ERR_CUDA = 0, 1, 2, 3
 PKV_ERR_TIMEOUT, PKV_ERR_BAD_TABLE, PKV_ERR_WORKSPACE = 4, 5, 6
 PKV_F32, PKV_BF16 = 0, 1
 PKV_DEVERR_BAD_PAGE, PKV_DEVERR_BAD_LEN, PKV_DEVERR_TIMEOUT = 0x1, 0x2, 0x4
+PKV_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 
@@ -40,6 +41,9 @@ _lib.paged_attn_workspace_size.argtypes = [_i, _i, _i, _i, _i]
 _lib.paged_attn.restype = _i
 _lib.paged_attn.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i,
                             _i, _f, _i, _vp, _vp, _sz, _vp]
+_lib.paged_decode_noalloc.restype = _i
+_lib.paged_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
+                                      _f, _vp, _vp]
 _lib.pkv_resolve.restype = _i
 _lib.pkv_resolve.argtypes = [ctypes.POINTER(ctypes.c_int32), _i, _i, _i,
                              ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]
@@ -97,6 +101,16 @@ def paged_attn(q, k_pages, v_pages, block_table, seq_lens, page_size, num_seqs, 
         _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens), page_size,
         num_seqs, q_len, H, H_kv, d, num_pages, max_pages_per_seq, max_seq_len, int(causal),
         float(scale), dtype, _ptr(out), _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def paged_decode_noalloc(q, k_pages, v_pages, block_table, seq_lens, page_size, num_seqs, H,
+                         H_kv, d, num_pages, max_pages_per_seq, max_seq_len, scale, out,
+                         stream=None):
+    """Decode with the library's static scratch (allocates nothing)."""
+    _check("paged_decode_noalloc", _lib.paged_decode_noalloc(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens), page_size,
+        num_seqs, H, H_kv, d, num_pages, max_pages_per_seq, max_seq_len, float(scale), _ptr(out),
+        _stream(stream)))
 
 
 def pkv_resolve(block_table_row, page_size: int, token: int):

@@ -18,7 +18,7 @@ CSRC = os.path.join(PKG, "csrc")
 ROOT = os.path.dirname(PKG)
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libpkv.so")
-SOURCES = ["pkv_api.cu", "decode.cu", "simt_fp32.cu", "prefill_sm100.cu"]
+SOURCES = ["pkv_api.cu", "decode.cu", "decode_noalloc.cu", "simt_fp32.cu", "prefill_sm100.cu"]
 HEADERS = ["common.cuh", "sm100_ptx.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

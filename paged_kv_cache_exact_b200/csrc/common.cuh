@@ -98,4 +98,7 @@ cudaError_t launch_decode_bf16(const DecodeParams& p, cudaStream_t stream);
 cudaError_t launch_simt_f32(const SimtParams& p, cudaStream_t stream);
 cudaError_t launch_prefill_bf16(const PrefillParams& p, cudaStream_t stream);
 
+// Device address of the library's error word on the current device.
+int device_error_word(unsigned int** out);
+
 }  // namespace pkv

@@ -47,6 +47,10 @@ int cuda_status(cudaError_t e) {
 
 }  // namespace
 
+namespace pkv {
+int device_error_word(unsigned int** out) { return error_word(out); }
+}  // namespace pkv
+
 extern "C" {
 
 const char* pkv_status_string(int status) {

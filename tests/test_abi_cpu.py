@@ -111,3 +111,16 @@ def test_attn_prefill_rejects_bad_arguments(args, status):
     *ptrs, Bn, H, N, d, causal, scale, dtype = args
     assert B.raw_status("attn_prefill", *ptrs, Bn, H, N, d, causal, ctypes.c_float(scale),
                         dtype, None) == status
+
+
+def test_no_alloc_decode_rejects_plans_beyond_its_scratch():
+    """A plan whose partials exceed PKV_NOALLOC_SCRATCH_BYTES is refused with
+    PKV_ERR_WORKSPACE before anything is launched."""
+    S, H, L, ps = 2048, 32, 8192, 16
+    assert B.paged_attn_workspace_size(S, H, 128, L, ps) > B.PKV_NOALLOC_SCRATCH_BYTES
+    st = B.raw_status("paged_decode_noalloc", FAKE, FAKE, FAKE, FAKE, FAKE, ps, S, H, H, 128,
+                      1 << 16, L // ps, L, ctypes.c_float(0.1), FAKE, None)
+    assert st == B.PKV_ERR_WORKSPACE
+    st = B.raw_status("paged_decode_noalloc", FAKE, FAKE, FAKE, FAKE, FAKE, ps, 4, H, H, 64,
+                      64, L // ps, L, ctypes.c_float(0.1), FAKE, None)
+    assert st == B.PKV_ERR_UNSUPPORTED
