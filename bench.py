@@ -43,7 +43,7 @@ WORKLOAD = ("serving step: causal prefill B=4 H=32 N=4096 d=128 bf16 + paged dec
             "32 heads d=128 bf16, seq_lens U[512,8192], page_size 16")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-PREFILL_SRC = ["prefill_sm100.cu", "sm100_ptx.cuh", "common.cuh"]
+PREFILL_SRC = ["prefill_sm100.cu", "sm100_ptx.cuh", "exp2_poly.cuh", "common.cuh"]
 DECODE_SRC = ["decode.cu", "common.cuh"]
 
 

@@ -17,7 +17,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 // exp2(-inf) = +0, which masked scores rely on.
 PKV_DEVINLINE float ex2(float x) {
   float y;
-  asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 

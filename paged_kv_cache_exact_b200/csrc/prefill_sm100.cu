@@ -14,7 +14,7 @@
 // * CTA = two 128-row Q tiles of one (batch, head) sharing every K/V tile.
 //   Warp roles: warps 0-3 and 4-7 are the softmax warpgroups of Q tile 0 and 1
 //   (one thread per row = one TMEM lane), warp 8 issues TMA loads, warp 9
-//   issues tcgen05.mma from one elected lane.
+//   issues tcgen05.mma from one elected lane, warps 10-11 only lend registers.
 // * TMEM (512 columns x 128 lanes x 32 bit): S0 | S1 | O0 | O1, 128 f32 columns
 //   each.  P (bf16) overwrites the first 64 columns of its S once the softmax
 //   has read S into registers, and feeds the PV product straight from TMEM
@@ -36,6 +36,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "exp2_poly.cuh"
 #include "sm100_ptx.cuh"
 
 namespace pkv {
@@ -48,11 +49,32 @@ constexpr int BM = 128;            // rows per Q tile
 constexpr int BN = 128;            // keys per K/V tile
 constexpr int kQTiles = 2;         // Q tiles per CTA
 constexpr int kStages = 2;         // K ring and V ring depth
-constexpr int kThreads = 320;      // 10 warps
+constexpr int kThreads = 384;      // 3 warpgroups: softmax 0, softmax 1, producer/MMA
+// Register split: launched at kLaunchRegs per thread (3 warps per SM
+// sub-partition -> at most 168), then the producer/MMA warpgroup drops to
+// kRegsSide and both softmax warpgroups rise to kRegsSoftmax.  The split must
+// add up to no more than the launch allocation or setmaxnreg.inc would wait
+// forever, so the host refuses to launch unless the kernel was built with
+// exactly kLaunchRegs registers.
+constexpr int kLaunchRegs = 168;
+constexpr int kRegsSoftmax = 208;
+constexpr int kRegsSide = 88;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsSide <= kThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
 constexpr int kTileBytes = BM * D * 2;             // 32 KB
 constexpr int kHalfBytes = kTileBytes / 2;         // one 64-column block: 16 KB
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 constexpr float kRescaleThreshold = 8.0f;          // log2 units
+// Softmax tuning: one exp2 pair in kPolyEvery goes to the FMA-pipe polynomial
+// (0 = all on MUFU); kSplitP hands P to the PV product in two halves.
+#ifndef PKV_POLY_EVERY
+#define PKV_POLY_EVERY 0
+#endif
+#ifndef PKV_SPLIT_P
+#define PKV_SPLIT_P 1
+#endif
+constexpr int kPolyEvery = PKV_POLY_EVERY;
+constexpr bool kSplitP = PKV_SPLIT_P != 0;
 
 // Shared memory map (offsets from a 1024-aligned base).
 constexpr int kOffQ = 0;
@@ -66,10 +88,11 @@ enum Bar {
   kBarVFull = kBarKEmpty + kStages,
   kBarVEmpty = kBarVFull + kStages,
   kBarSFull = kBarVEmpty + kStages,   // + q tile
-  kBarPFull = kBarSFull + kQTiles,
+  kBarPHalf = kBarSFull + kQTiles,   // first 64 keys of P in TMEM (+ q tile)
+  kBarPFull = kBarPHalf + kQTiles,    // all of P in TMEM
   kBarODone = kBarPFull + kQTiles,
   kBarVFixed = kBarODone + kQTiles,   // last paged V tile after tail rows are zeroed
-  kBarDrain = kBarVFixed + 1,
+  kBarDrain = kBarVFixed + 1,         // abort path: wait for issued MMAs
   kNumBars = kBarDrain + 1
 };
 constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
@@ -90,18 +113,20 @@ struct Geometry {
 
 __device__ __forceinline__ Geometry cta_geometry(const PrefillParams& p) {
   Geometry g;
-  const int bh = blockIdx.x;
+  // grid.x walks the Q blocks of one (batch, head), heaviest causal block
+  // first, so the CTAs sharing a head's K/V run together and hit L2.
+  const int bh = blockIdx.y;
   g.b = bh / p.H;
   g.h = bh % p.H;
   g.kvh = g.h / (p.H / p.H_kv);
-  g.q0 = (gridDim.y - 1 - blockIdx.y) * (BM * kQTiles);   // heaviest causal blocks first
+  g.q0 = (gridDim.x - 1 - blockIdx.x) * (BM * kQTiles);
   g.q_len = p.q_len;
   int kv_len = p.kv_len;
   if (p.paged) {
     kv_len = p.seq_lens[g.b];
     const int cap = min(p.max_seq_len, p.max_pages * p.page_size);
     if (kv_len < p.q_len || kv_len > cap) {
-      if (blockIdx.y == 0 && g.h == 0 && threadIdx.x == 0) flag_error(p.err, PKV_DEVERR_BAD_LEN);
+      if (blockIdx.x == 0 && g.h == 0 && threadIdx.x == 0) flag_error(p.err, PKV_DEVERR_BAD_LEN);
       kv_len = max(0, min(kv_len, cap));
     }
   }
@@ -136,7 +161,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumBars; ++i) {
-      const uint32_t cnt = (i == kBarPFull || i == kBarPFull + 1) ? 128u : 1u;
+      // P halves: one arrival per softmax thread; everything else: one arrival.
+      const bool per_thread = (i >= kBarPHalf && i < kBarPFull + kQTiles);
+      const uint32_t cnt = per_thread ? 128u : 1u;
       mbar_init(bar(i), cnt);
     }
     *abort_flag = 0;
@@ -163,6 +190,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
     return true;
   };
+
+  if (warp >= 8) regs_decrease<kRegsSide>();
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer --
@@ -259,75 +288,108 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
   } else if (warp == 9) {
     // ----------------------------------------------------------------- MMA --
-    if (lane == 0 && n > 0) {
-      const uint32_t sQ = sbase + kOffQ;
+    // Issue order per K/V tile j: PV0(j) S0(j+1) PV1(j) S1(j+1).  The softmax of
+    // one Q tile then overlaps the other tile's MMAs (ping-pong), and each
+    // S_t(j+1) is issued after PV_t(j), which consumes the P_t(j) it overwrites
+    // (tcgen05.mma executes in issue order).  Descriptors are precomputed per
+    // stage so that an issue costs one add and the MMA: a 128x128x16 MMA
+    // retires in 64 cycles, less than a descriptor rebuild takes.  The warp
+    // runs converged and one elected lane issues.
+    auto wwait = [&](int b, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, wait(b, parity));
+    };
+    if (n > 0) {
       const bool last_fix = kPaged && (g.kv_len - (n - 1) * BN) < BN;
+      const uint64_t dq0 = make_sdesc(sbase + kOffQ, 16, 1024);
+      const uint64_t dq1 = make_sdesc(sbase + kOffQ + kTileBytes, 16, 1024);
+      const uint64_t dk0 = make_sdesc(sbase + kOffK, 16, 1024);
+      const uint64_t dk1 = make_sdesc(sbase + kOffK + kTileBytes, 16, 1024);
+      const uint64_t dv0 = make_sdesc(sbase + kOffV, kHalfBytes, 1024);
+      const uint64_t dv1 = make_sdesc(sbase + kOffV + kTileBytes, kHalfBytes, 1024);
+      const bool leader = elect_one();
       auto issue_s = [&](int t, int j) {
-        const int st = j % kStages;
-        const uint32_t sK = sbase + kOffK + st * kTileBytes;
+        const uint64_t dk = (j % kStages) ? dk1 : dk0;
+        const uint64_t dq = t ? dq1 : dq0;
+        const uint32_t tS = tmem + kColS + 128 * t;
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (kk / 4) * kHalfBytes + (kk % 4) * 32;
-          const uint64_t da = make_sdesc(sQ + t * kTileBytes + koff, 16, 1024);
-          const uint64_t db = make_sdesc(sK + koff, 16, 1024);
-          mma_ss(tmem + kColS + 128 * t, da, db, kIdescS, kk > 0);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t koff = ((kk / 4) * kHalfBytes + (kk % 4) * 32) >> 4;
+            mma_ss(tS, dq + koff, dk + koff, kIdescS, kk > 0);
+          }
+          mma_commit(bar(kBarSFull + t));
         }
-        mma_commit(bar(kBarSFull + t));
+        __syncwarp();
       };
-      auto issue_pv = [&](int t, int j) {
-        const int st = j % kStages;
-        const uint32_t sV = sbase + kOffV + st * kTileBytes;
+      // O_t += P_t V over key steps [kk0, kk0 + 4): P arrives in two halves.
+      auto issue_pv_half = [&](int t, int j, int kk0) {
+        const uint64_t dv = (j % kStages) ? dv1 : dv0;
+        const uint32_t tS = tmem + kColS + 128 * t;
+        const uint32_t tO = tmem + kColO + 128 * t;
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t db = make_sdesc(sV + kk * 16 * 128, kHalfBytes, 1024);
-          mma_ts(tmem + kColO + 128 * t, tmem + kColS + 128 * t + kk * 8, db, kIdescO,
-                 (j > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = kk0; kk < kk0 + BN / 32; ++kk)
+            mma_ts(tO, tS + kk * 8, dv + ((kk * 16 * 128) >> 4), kIdescO,
+                   (j > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(bar(kBarODone + t));
+        __syncwarp();
       };
-      bool ok = wait(kBarQ, 0) && wait(kBarKFull + 0, 0);
+      auto issue_pv = [&](int t, int j) -> bool {
+        if (kSplitP) {
+          if (!wwait(kBarPHalf + t, j & 1)) return false;
+          tc_fence_after();
+          issue_pv_half(t, j, 0);
+        }
+        if (!wwait(kBarPFull + t, j & 1)) return false;
+        tc_fence_after();
+        if (!kSplitP) issue_pv_half(t, j, 0);
+        issue_pv_half(t, j, BN / 32);
+        if (leader) mma_commit(bar(kBarODone + t));
+        __syncwarp();
+        return true;
+      };
+      auto commit = [&](int b) {
+        if (leader) mma_commit(bar(b));
+        __syncwarp();
+      };
+      bool ok = wwait(kBarQ, 0) && wwait(kBarKFull + 0, 0);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
         issue_s(1, 0);
-        mma_commit(bar(kBarKEmpty + 0));
+        commit(kBarKEmpty + 0);
       }
       for (int j = 0; j < n && ok; ++j) {
         const int st = j % kStages;
-        const uint32_t ph = (j / kStages) & 1;
         if (last_fix && j == n - 1)
-          ok = wait(kBarVFixed, 0);
+          ok = wwait(kBarVFixed, 0);
         else
-          ok = wait(kBarVFull + st, ph);
-        ok = ok && wait(kBarPFull + 0, j & 1);
+          ok = wwait(kBarVFull + st, (j / kStages) & 1);
+        ok = ok && issue_pv(0, j);
         if (!ok) break;
-        tc_fence_after();
-        issue_pv(0, j);
         if (j + 1 < n) {
-          const int st1 = (j + 1) % kStages;
-          ok = wait(kBarKFull + st1, ((j + 1) / kStages) & 1);
+          ok = wwait(kBarKFull + (j + 1) % kStages, ((j + 1) / kStages) & 1);
           if (!ok) break;
           tc_fence_after();
           issue_s(0, j + 1);
         }
-        ok = wait(kBarPFull + 1, j & 1);
+        ok = issue_pv(1, j);
         if (!ok) break;
-        tc_fence_after();
-        issue_pv(1, j);
-        mma_commit(bar(kBarVEmpty + st));
+        commit(kBarVEmpty + st);
         if (j + 1 < n) {
           issue_s(1, j + 1);
-          mma_commit(bar(kBarKEmpty + (j + 1) % kStages));
+          commit(kBarKEmpty + (j + 1) % kStages);
         }
       }
       if (!ok) {
         // Let every MMA already issued finish before TMEM is released.
-        mma_commit(bar(kBarDrain));
+        commit(kBarDrain);
         mbar_wait_bounded(bar(kBarDrain), 0, kWaitLimitNs);
       }
     }
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------------- softmax --
+    regs_increase<kRegsSoftmax>();
     const int t = warp >> 2;                         // Q tile of this warpgroup
     const int r = threadIdx.x & 127;                 // row in tile = TMEM lane
     const int row = g.q0 + t * BM + r;               // query row
@@ -354,18 +416,26 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       tmem_wait_ld();
       const int k0 = j * BN;
-      float mx = -INFINITY;
-      if (k0 + BN - 1 > limit) {                     // diagonal or tail tile: mask
+      const bool masked = k0 + BN - 1 > limit;       // diagonal or tail tile
+      if (masked) {
 #pragma unroll
-        for (int i = 0; i < 128; ++i) {
-          const float v = (k0 + i <= limit) ? __uint_as_float(s[i]) : -INFINITY;
-          s[i] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 128; ++i) mx = fmaxf(mx, __uint_as_float(s[i]));
+        for (int i = 0; i < 128; ++i)
+          if (k0 + i > limit) s[i] = __float_as_uint(-INFINITY);
       }
+      // row max: eight chains of 3-input max (dependency depth 8)
+      float am[8];
+#pragma unroll
+      for (int a = 0; a < 8; ++a) am[a] = __uint_as_float(s[a]);
+#pragma unroll
+      for (int i = 8; i + 16 <= 128; i += 16) {        // elements 8 .. 119
+#pragma unroll
+        for (int a = 0; a < 8; ++a)
+          am[a] = max3(am[a], __uint_as_float(s[i + 2 * a]), __uint_as_float(s[i + 2 * a + 1]));
+      }
+#pragma unroll
+      for (int a = 0; a < 8; ++a) am[a] = fmaxf(am[a], __uint_as_float(s[120 + a]));   // 120 .. 127
+      const float mx = max3(max3(am[0], am[1], am[2]), max3(am[3], am[4], am[5]),
+                            fmaxf(am[6], am[7]));
       const float m_tile = mx * c;                  // running max in log2 units
       float alpha = 1.f;
       bool rescale = false;
@@ -375,19 +445,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         rescale = true;
       }
       const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
-      float rowsum = 0.f;
-#pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {            // 64 scores -> 32 packed bf16 pairs
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2(fmaf(__uint_as_float(s[64 * ch + 2 * i]), c, neg_m));
-          const float p1 = ex2(fmaf(__uint_as_float(s[64 * ch + 2 * i + 1]), c, neg_m));
-          rowsum += p0 + p1;
-          pk[i] = pack_bf16x2(p0, p1);
-        }
-        tmem_st32(tS + 32 * ch, pk);
-      }
+      // O must be rescaled before PV(j) may start, i.e. before any P is handed over.
       if (__any_sync(0xffffffffu, rescale) && j > 0) {   // alpha = 1 in rows that keep m
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
@@ -399,7 +457,42 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           tmem_st32(tO + 32 * ch, o);
         }
       }
-      l = l * alpha + rowsum;
+      // Masked tiles stay on MUFU (exact zeros); elsewhere one pair in four
+      // takes the FMA-pipe polynomial.
+      const bool poly = !__any_sync(0xffffffffu, masked);
+      const uint64_t c2 = f2(c, c), nm2 = f2(neg_m, neg_m);
+      uint64_t acc[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) acc[a] = f2(0.f, 0.f);
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {            // 64 scores -> 32 packed bf16 pairs
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int e = 64 * ch + 2 * i;
+          const uint64_t x2 = fma2(f2(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), c2, nm2);
+          float p0, p1;
+          if (kPolyEvery > 0 && poly && (i % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
+            exp2_poly_pair(x2, p0, p1);
+          } else {
+            float x0, x1;
+            unf2(x2, x0, x1);
+            p0 = ex2(x0);
+            p1 = ex2(x1);
+          }
+          acc[i & 3] = add2(acc[i & 3], f2(p0, p1));
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(tS + 32 * ch, pk);
+        if (kSplitP && ch == 0) {                  // first half of P: PV(j) may start
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar(kBarPHalf + t));
+        }
+      }
+      float s0, s1;
+      unf2(add2(add2(acc[0], acc[1]), add2(acc[2], acc[3])), s0, s1);
+      l = l * alpha + (s0 + s1);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(kBarPFull + t));
@@ -485,8 +578,13 @@ cudaError_t set_smem_attr() {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<kPaged>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  // The in-kernel register split assumes this exact launch allocation.
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, prefill_kernel<kPaged>);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != kLaunchRegs) return cudaErrorNotSupported;
+  e = cudaFuncSetAttribute(prefill_kernel<kPaged>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kSmemBytes);
   if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = 1;
   return e;
 }
@@ -514,8 +612,8 @@ cudaError_t launch_prefill_bf16(const PrefillParams& p, cudaStream_t stream) {
       return cudaErrorInvalidValue;
   }
   const int m_blocks = (p.q_len + BM * kQTiles - 1) / (BM * kQTiles);
-  if (m_blocks > 65535) return cudaErrorNotSupported;
-  dim3 grid((unsigned)p.B * p.H, m_blocks);
+  if ((long long)p.B * p.H > 65535) return cudaErrorNotSupported;
+  dim3 grid(m_blocks, (unsigned)p.B * p.H);
   cudaError_t e;
   if (p.paged) {
     e = set_smem_attr<true>();
