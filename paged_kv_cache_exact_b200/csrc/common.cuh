@@ -88,6 +88,7 @@ struct PrefillParams {
   int paged, page_size, page_shift, num_pages, max_pages, max_seq_len;
   int causal;
   float scale_log2;
+  int head_group;   // (batch, head) pairs scheduled together (set by the launcher)
 };
 
 // Split plan for decode: fixed-size key chunks per (sequence, head).

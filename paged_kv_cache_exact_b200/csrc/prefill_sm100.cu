@@ -66,7 +66,8 @@ constexpr int kHalfBytes = kTileBytes / 2;         // one 64-column block: 16 KB
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 constexpr float kRescaleThreshold = 8.0f;          // log2 units
 // Softmax tuning: one exp2 pair in kPolyEvery goes to the FMA-pipe polynomial
-// (0 = all on MUFU); kSplitP hands P to the PV product in two halves.
+// (0 = all on MUFU; measured slower at 1/8, 1/4 and 1/2, so off); kSplitP
+// hands P to the PV product in two halves.
 #ifndef PKV_POLY_EVERY
 #define PKV_POLY_EVERY 0
 #endif
@@ -74,6 +75,13 @@ constexpr float kRescaleThreshold = 8.0f;          // log2 units
 #define PKV_SPLIT_P 1
 #endif
 constexpr int kPolyEvery = PKV_POLY_EVERY;
+// Start the first half's exponentials against the current reference max while
+// the row max is reduced (redo rows whose max grew past the threshold).
+// Measured: +2.5% on the 4x32x4096 prefill, -5..15% on the 32K paged prefill.
+#ifndef PKV_SPEC_EXP
+#define PKV_SPEC_EXP 0
+#endif
+constexpr bool kSpeculativeExp = PKV_SPEC_EXP != 0;
 constexpr bool kSplitP = PKV_SPLIT_P != 0;
 
 // Shared memory map (offsets from a 1024-aligned base).
@@ -113,20 +121,30 @@ struct Geometry {
 
 __device__ __forceinline__ Geometry cta_geometry(const PrefillParams& p) {
   Geometry g;
-  // grid.x walks the Q blocks of one (batch, head), heaviest causal block
-  // first, so the CTAs sharing a head's K/V run together and hit L2.
-  const int bh = blockIdx.y;
+  // 1-D grid, scheduled in groups of p.head_group (batch, head) pairs: within
+  // a group the heaviest causal Q block of every head comes first, then the
+  // next heaviest, ...  The host sizes a group so that its K/V (about 32 MB)
+  // stays in L2 while its Q blocks run; the lightest blocks fill the tail.
+  const int m_blocks = (p.q_len + BM * kQTiles - 1) / (BM * kQTiles);
+  const int BH = p.B * p.H;
+  const int hg = p.head_group;
+  const int per_group = hg * m_blocks;
+  const int group = blockIdx.x / per_group;
+  const int r = blockIdx.x - group * per_group;
+  const int heads_here = min(hg, BH - group * hg);
+  const int rank = r / heads_here;                  // 0 = heaviest Q block
+  const int bh = group * hg + (r - rank * heads_here);
   g.b = bh / p.H;
   g.h = bh % p.H;
   g.kvh = g.h / (p.H / p.H_kv);
-  g.q0 = (gridDim.x - 1 - blockIdx.x) * (BM * kQTiles);
+  g.q0 = (m_blocks - 1 - rank) * (BM * kQTiles);
   g.q_len = p.q_len;
   int kv_len = p.kv_len;
   if (p.paged) {
     kv_len = p.seq_lens[g.b];
     const int cap = min(p.max_seq_len, p.max_pages * p.page_size);
     if (kv_len < p.q_len || kv_len > cap) {
-      if (blockIdx.x == 0 && g.h == 0 && threadIdx.x == 0) flag_error(p.err, PKV_DEVERR_BAD_LEN);
+      if (g.q0 == 0 && g.h == 0 && threadIdx.x == 0) flag_error(p.err, PKV_DEVERR_BAD_LEN);
       kv_len = max(0, min(kv_len, cap));
     }
   }
@@ -436,37 +454,17 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       for (int a = 0; a < 8; ++a) am[a] = fmaxf(am[a], __uint_as_float(s[120 + a]));   // 120 .. 127
       const float mx = max3(max3(am[0], am[1], am[2]), max3(am[3], am[4], am[5]),
                             fmaxf(am[6], am[7]));
-      const float m_tile = mx * c;                  // running max in log2 units
-      float alpha = 1.f;
-      bool rescale = false;
-      if (m_tile > m_ref + kRescaleThreshold || (m_ref == -INFINITY && m_tile != -INFINITY)) {
-        alpha = ex2(m_ref - m_tile);               // m_ref = -inf -> 0
-        m_ref = m_tile;
-        rescale = true;
-      }
-      const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
-      // O must be rescaled before PV(j) may start, i.e. before any P is handed over.
-      if (__any_sync(0xffffffffu, rescale) && j > 0) {   // alpha = 1 in rows that keep m
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t o[32];
-          tmem_ld32(tO + 32 * ch, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tO + 32 * ch, o);
-        }
-      }
-      // Masked tiles stay on MUFU (exact zeros); elsewhere one pair in four
-      // takes the FMA-pipe polynomial.
+      // The first half's exponentials are computed against the current
+      // reference max while the row max above is still being reduced (the two
+      // are independent, so they interleave); they are redone only in rows
+      // whose max grew past the rescale threshold, which after the first tile
+      // is rare.  Masked tiles stay on MUFU (exact zeros); elsewhere
+      // kPolyEvery selects the share of pairs on the FMA-pipe polynomial.
       const bool poly = !__any_sync(0xffffffffu, masked);
-      const uint64_t c2 = f2(c, c), nm2 = f2(neg_m, neg_m);
+      const uint64_t c2 = f2(c, c);
       uint64_t acc[4];
-#pragma unroll
-      for (int a = 0; a < 4; ++a) acc[a] = f2(0.f, 0.f);
-#pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {            // 64 scores -> 32 packed bf16 pairs
-        uint32_t pk[32];
+      auto exp_half = [&](int ch, float neg_m, uint32_t (&pk)[32]) {
+        const uint64_t nm2 = f2(neg_m, neg_m);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const int e = 64 * ch + 2 * i;
@@ -483,13 +481,48 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           acc[i & 3] = add2(acc[i & 3], f2(p0, p1));
           pk[i] = pack_bf16x2(p0, p1);
         }
-        tmem_st32(tS + 32 * ch, pk);
-        if (kSplitP && ch == 0) {                  // first half of P: PV(j) may start
-          tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(bar(kBarPHalf + t));
+      };
+#pragma unroll
+      for (int a = 0; a < 4; ++a) acc[a] = f2(0.f, 0.f);
+      uint32_t pk[32];
+      if (kSpeculativeExp) exp_half(0, (m_ref == -INFINITY) ? 0.f : -m_ref, pk);
+      const float m_tile = mx * c;                  // running max in log2 units
+      float alpha = 1.f;
+      bool rescale = false;
+      if (m_tile > m_ref + kRescaleThreshold || (m_ref == -INFINITY && m_tile != -INFINITY)) {
+        alpha = ex2(m_ref - m_tile);               // m_ref = -inf -> 0
+        m_ref = m_tile;
+        rescale = true;
+      }
+      const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+      if (!kSpeculativeExp) exp_half(0, neg_m, pk);
+      if (__any_sync(0xffffffffu, rescale)) {
+        if (kSpeculativeExp && rescale) {          // redo this row's first half
+#pragma unroll
+          for (int a = 0; a < 4; ++a) acc[a] = f2(0.f, 0.f);
+          exp_half(0, neg_m, pk);
+        }
+        // O must be rescaled before PV(j) may start, i.e. before any P is handed over.
+        if (j > 0) {                               // alpha = 1 in rows that keep m
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * ch, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tO + 32 * ch, o);
+          }
         }
       }
+      tmem_st32(tS, pk);
+      if (kSplitP) {                               // first half of P: PV(j) may start
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(kBarPHalf + t));
+      }
+      exp_half(1, neg_m, pk);
+      tmem_st32(tS + 32, pk);
       float s0, s1;
       unf2(add2(add2(acc[0], acc[1]), add2(acc[2], acc[3])), s0, s1);
       l = l * alpha + (s0 + s1);
@@ -611,18 +644,30 @@ cudaError_t launch_prefill_bf16(const PrefillParams& p, cudaStream_t stream) {
         !encode_3d(&tv, p.V, D, p.kv_len, bhkv, row_bytes, row_bytes * p.kv_len, BN, 1))
       return cudaErrorInvalidValue;
   }
-  const int m_blocks = (p.q_len + BM * kQTiles - 1) / (BM * kQTiles);
-  if ((long long)p.B * p.H > 65535) return cudaErrorNotSupported;
-  dim3 grid(m_blocks, (unsigned)p.B * p.H);
+  const long long m_blocks = (p.q_len + BM * kQTiles - 1) / (BM * kQTiles);
+  const long long ctas = m_blocks * p.B * p.H;
+  if (ctas > 0x7fffffffLL) return cudaErrorNotSupported;
+  dim3 grid((unsigned)ctas);
+  // Heads scheduled together: as many as keep about 32 MB of K/V live in L2
+  // (query heads sharing a kv head count once).
+  PrefillParams q = p;
+  {
+    const long long kv_len = p.paged ? p.max_seq_len : p.kv_len;
+    const long long kv_bytes = 2LL * kv_len * D * 2;              // K and V of one kv head
+    const int group_q = p.H / p.H_kv;
+    long long hg = (32LL << 20) / (kv_bytes > 0 ? kv_bytes : 1) * group_q;
+    hg = hg < 1 ? 1 : (hg > 32 ? 32 : hg);
+    q.head_group = (int)hg;
+  }
   cudaError_t e;
   if (p.paged) {
     e = set_smem_attr<true>();
     if (e != cudaSuccess) return e;
-    prefill_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, p);
+    prefill_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, q);
   } else {
     e = set_smem_attr<false>();
     if (e != cudaSuccess) return e;
-    prefill_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, p);
+    prefill_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, q);
   }
   return cudaGetLastError();
 }
