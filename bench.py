@@ -277,6 +277,7 @@ def run_gpu(args, rank, world, dist):
     barrier()
     e2e_ms = e0.elapsed_time(e1) / n_e2e
 
+    append = measure_append(device, stream, peaks)
     total_ms, e2e_ms, pre_ms, dec_ms = reduce_max([total_ms, e2e_ms, pre_ms, dec_ms], dist,
                                                   device)
     ms_step = total_ms / args.steps
@@ -314,10 +315,56 @@ def run_gpu(args, rank, world, dist):
                 "d2h_bytes_per_step": meta["d2h"], "ms_per_step": e2e_ms,
                 "note": "pinned host Q/K/V, q, block_table, seq_lens in and O, out back every "
                         "step; the KV page pool is resident device state"},
+        "append": append,
         "gpu_launches": args.steps * meta["launches_per_step"],
         "clocks": clocks,
     }
     return line, meta["inputs"]
+
+
+def append_setup(device, seqs=64, tokens=512, page_size=16, H_kv=32, d=128):
+    """A prefill-sized KV append (every sequence writes `tokens` new rows into
+    shuffled pages of its own pool); inputs and pool exceed L2."""
+    import torch
+
+    gen = torch.Generator().manual_seed(1099)
+    rows = seqs * tokens
+    pages_per = tokens // page_size
+    num_pages = seqs * pages_per
+    k_new = torch.randn(rows, H_kv, d, generator=gen).to(torch.bfloat16).to(device)
+    v_new = torch.randn(rows, H_kv, d, generator=gen).to(torch.bfloat16).to(device)
+    perm = torch.randperm(num_pages, generator=gen).to(torch.int32)
+    table = perm.view(seqs, pages_per).contiguous().to(device)
+    cu = (torch.arange(seqs + 1, dtype=torch.int32) * tokens).to(device)
+    start = torch.zeros(seqs, dtype=torch.int32, device=device)
+    k_pages = torch.empty(num_pages, page_size, H_kv, d, dtype=torch.bfloat16, device=device)
+    v_pages = torch.empty_like(k_pages)
+    from paged_kv_cache_exact_b200 import binding as B
+
+    def run(stream):
+        B.paged_kv_append(k_new, v_new, cu, start, table, pages_per, seqs, rows, k_pages, v_pages,
+                          num_pages, page_size, H_kv, d, B.PKV_BF16, stream)
+    moved = 2 * 2 * rows * H_kv * d * 2           # read K,V rows + write them
+    return run, moved, f"{seqs} seqs x {tokens} new tokens, H_kv={H_kv} d={d} bf16, page 16"
+
+
+def measure_append(device, stream, peaks, iters=50):
+    import torch
+
+    run, moved, desc = append_setup(device)
+    for _ in range(3):
+        run(stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    e0.record(stream)
+    for _ in range(iters):
+        run(stream)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = e0.elapsed_time(e1) / iters
+    gbs = moved / (ms / 1e3) / 1e9
+    return {"workload": desc, "ms": ms, "gbs": gbs, "frac": gbs / peaks["hbm_gbs"],
+            "bytes": moved, "note": "paged_kv_append timed alone after the step loop; not in value"}
 
 
 # ---------------------------------------------------------------------------
@@ -430,6 +477,7 @@ PROFILE_CASES = {
     "paged-prefill": "paged causal prefill 1x32x32768x128, 128 shuffled pages of 256",
     "decode16": "paged decode, 16 seqs x 32 heads, seq_lens U[512,8192], page_size 16 "
                 "(the step's decode distribution, a quarter of the sequences)",
+    "append": "paged KV append, 64 seqs x 512 new tokens, H_kv=32 d=128 bf16, page 16",
 }
 
 
@@ -439,6 +487,14 @@ def run_profile(args):
     from paged_kv_cache_exact_b200 import api
     from paged_kv_cache_exact_b200.workloads import make_paged, workload
     dev = torch.device("cuda", 0)
+    if args.profile == "append":
+        run, moved, desc = append_setup(dev)
+        for _ in range(args.steps):
+            run(None)
+        torch.cuda.synchronize(dev)
+        print(json.dumps({"profile": "append", "case": desc, "iterations": args.steps,
+                          "bytes_per_launch": moved}))
+        return
     if args.profile == "prefill":
         w = workload(2)
         Q, K, V = w.Q.to(dev), w.K.to(dev), w.V.to(dev)

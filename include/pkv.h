@@ -64,7 +64,8 @@ typedef enum {
   PKV_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
   PKV_ERR_TIMEOUT = 4,       /* device: a pipeline wait gave up (pkv_last_device_error) */
   PKV_ERR_BAD_TABLE = 5,     /* device: a page id or sequence length was out of range */
-  PKV_ERR_WORKSPACE = 6      /* workspace missing or smaller than paged_attn_workspace_size() */
+  PKV_ERR_WORKSPACE = 6,     /* workspace missing or smaller than paged_attn_workspace_size() */
+  PKV_ERR_OUT_OF_PAGES = 7   /* allocator: not enough free pages (nothing was changed) */
 } pkv_status;
 
 typedef enum { PKV_F32 = 0, PKV_BF16 = 1 } pkv_dtype;
@@ -182,6 +183,98 @@ PKV_API int paged_decode_noalloc(const void* q, const void* k_pages, const void*
                                  int page_size, int num_seqs, int H, int H_kv, int d,
                                  int num_pages, int max_pages_per_seq, int max_seq_len,
                                  float scale, void* out, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* The write side of the paged cache.                                       */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * paged_kv_append - write new tokens' K and V rows into their pages.
+ *
+ * Defines: "Flash Attention: Fast, Memory-Efficient Attention for LLMs",
+ * section "KV Cache" (each decode step appends the new K_t, V_t; prefill
+ * stores the K/V of every prompt token), with the address of token position
+ * pos of sequence s given by "What is Paged FlashAttention?", "Practical
+ * example": page block_table[s][pos / page_size], offset pos % page_size.
+ *
+ * k_new, v_new : device, [num_new, H_kv, d]: rows of all sequences' new tokens,
+ *                sequence by sequence.
+ * cu_new       : device int32 [num_seqs + 1], non-decreasing, cu_new[0] = 0,
+ *                cu_new[num_seqs] = num_new: sequence s owns rows
+ *                [cu_new[s], cu_new[s+1]).
+ * start_pos    : device int32 [num_seqs]: position of sequence s's first new
+ *                token (its length before the append).
+ * block_table  : device int32 [num_seqs, max_pages_per_seq]; the pages covering
+ *                the new positions must already be allocated (pkv_alloc_reserve).
+ * k_pages,
+ * v_pages      : device, [num_pages, page_size, H_kv, d], written in place.
+ * dtype        : PKV_BF16 or PKV_F32; d is 64 or 128.
+ * A row whose page id is outside [0, num_pages) or whose position is past the
+ * table is skipped and flagged (PKV_DEVERR_BAD_PAGE / PKV_DEVERR_BAD_LEN).
+ * Rows must not target the same slot twice in one call.
+ */
+PKV_API int paged_kv_append(const void* k_new, const void* v_new, const int32_t* cu_new,
+                            const int32_t* start_pos, const int32_t* block_table,
+                            int max_pages_per_seq, int num_seqs, int num_new, void* k_pages,
+                            void* v_pages, int num_pages, int page_size, int H_kv, int d,
+                            int dtype, void* stream);
+
+/*
+ * paged_kv_copy_pages - copy whole pages (K and V): page src[i] -> page dst[i].
+ *
+ * Defines the copy half of copy-on-write ("FlashAttention and PagedAttention:
+ * Two Fixes for Two Different Bottlenecks", section "PagedAttention ... How it
+ * works": sequences share prefix blocks and copy only when they diverge).
+ * src, dst : device int32 [n]; ids in [0, num_pages) (others are skipped and
+ *            flagged); a dst must not also be a src in the same call.
+ */
+PKV_API int paged_kv_copy_pages(void* k_pages, void* v_pages, const int32_t* src,
+                                const int32_t* dst, int n, int num_pages, int page_size,
+                                int H_kv, int d, int dtype, void* stream);
+
+/*
+ * pkv_alloc_* - host page allocator (bookkeeping only; host memory).
+ *
+ * Defines: "FlashAttention and PagedAttention: Two Fixes for Two Different
+ * Bottlenecks", section "PagedAttention ... How it works" (fixed-size blocks,
+ * per-sequence block table, allocation on demand, shared prefixes with
+ * copy-on-write) and "Flash Attention: Fast, Memory-Efficient Attention for
+ * LLMs", section "PagedAttention (vLLM)" (pages of finished sequences are
+ * freed and reused).  Policy: the smallest free page id is handed out first;
+ * pages carry reference counts; only a shared, partially filled last page is
+ * ever copied, just before the sequence writes into it.  Not thread-safe.
+ *
+ * pkv_alloc_create    : pool of num_pages pages of page_size tokens; tables
+ *                       hold at most max_pages_per_seq pages.  NULL on error.
+ * pkv_alloc_add_seq   : register an empty sequence under seq_id.
+ * pkv_alloc_reserve   : grow seq_id by n_tokens.  *start_pos gets the position
+ *                       of its first new token.  If its partially filled last
+ *                       page is shared, that page is replaced by a fresh one
+ *                       and the copy the caller must run first (with
+ *                       paged_kv_copy_pages) is returned in *cow_src ->
+ *                       *cow_dst with *n_cow = 1 (else *n_cow = 0).
+ *                       PKV_ERR_OUT_OF_PAGES leaves everything unchanged.
+ * pkv_alloc_fork      : child_id shares all of parent_id's pages (same length).
+ * pkv_alloc_free_seq  : drop seq_id; pages nobody else holds return to the pool.
+ * pkv_alloc_seq_len   : current length of seq_id.
+ * pkv_alloc_block_table: host arrays table [n][max_pages_per_seq] (-1 padded)
+ *                       and seq_lens [n] for the n listed sequences.
+ * pkv_alloc_num_free  : free pages (-1 for NULL).
+ * pkv_alloc_page_refs : reference count of a page (-1 if out of range).
+ */
+typedef struct pkv_allocator pkv_allocator;
+PKV_API pkv_allocator* pkv_alloc_create(int num_pages, int page_size, int max_pages_per_seq);
+PKV_API void pkv_alloc_destroy(pkv_allocator* a);
+PKV_API int pkv_alloc_add_seq(pkv_allocator* a, int seq_id);
+PKV_API int pkv_alloc_reserve(pkv_allocator* a, int seq_id, int n_tokens, int32_t* start_pos,
+                              int32_t* cow_src, int32_t* cow_dst, int* n_cow);
+PKV_API int pkv_alloc_fork(pkv_allocator* a, int parent_id, int child_id);
+PKV_API int pkv_alloc_free_seq(pkv_allocator* a, int seq_id);
+PKV_API int pkv_alloc_seq_len(const pkv_allocator* a, int seq_id, int* len);
+PKV_API int pkv_alloc_block_table(const pkv_allocator* a, const int* seq_ids, int n,
+                                  int32_t* table, int32_t* seq_lens);
+PKV_API int pkv_alloc_num_free(const pkv_allocator* a);
+PKV_API int pkv_alloc_page_refs(const pkv_allocator* a, int page);
 
 /*
  * pkv_resolve - host-side page-table address resolution (for tests and tools).

@@ -91,6 +91,29 @@ struct PrefillParams {
   int head_group;   // (batch, head) pairs scheduled together (set by the launcher)
 };
 
+struct AppendParams {
+  const void* k_new;           // [num_new, H_kv, d]
+  const void* v_new;
+  const int32_t* cu_new;       // [num_seqs + 1]
+  const int32_t* start_pos;    // [num_seqs]
+  const int32_t* block_table;  // [num_seqs, max_pages]
+  void* k_pages;               // [P, ps, H_kv, d]
+  void* v_pages;
+  unsigned int* err;
+  int num_seqs, num_new, max_pages, num_pages, page_size, page_shift;
+  size_t row_bytes;            // H_kv * d * element size
+};
+
+struct CopyPagesParams {
+  void* k_pages;
+  void* v_pages;
+  const int32_t* src;
+  const int32_t* dst;
+  unsigned int* err;
+  int n, num_pages;
+  size_t page_bytes;           // page_size * H_kv * d * element size
+};
+
 // Split plan for decode: fixed-size key chunks per (sequence, head).
 void decode_plan(int num_seqs, int H, int max_seq_len, int page_size,
                  int* split_tokens, int* max_splits);
@@ -98,6 +121,8 @@ void decode_plan(int num_seqs, int H, int max_seq_len, int page_size,
 cudaError_t launch_decode_bf16(const DecodeParams& p, cudaStream_t stream);
 cudaError_t launch_simt_f32(const SimtParams& p, cudaStream_t stream);
 cudaError_t launch_prefill_bf16(const PrefillParams& p, cudaStream_t stream);
+cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
+cudaError_t launch_copy_pages(const CopyPagesParams& p, cudaStream_t stream);
 
 // Device address of the library's error word on the current device.
 int device_error_word(unsigned int** out);

@@ -62,6 +62,7 @@ const char* pkv_status_string(int status) {
     case PKV_ERR_TIMEOUT: return "device pipeline wait timed out";
     case PKV_ERR_BAD_TABLE: return "page id or sequence length out of range";
     case PKV_ERR_WORKSPACE: return "workspace missing or too small";
+    case PKV_ERR_OUT_OF_PAGES: return "no free pages left in the pool";
     default: return "unknown status";
   }
 }
@@ -204,6 +205,50 @@ int paged_attn(const void* q, const void* k_pages, const void* v_pages,
   p.causal = causal;
   p.scale_log2 = scale * pkv::kLog2e;
   return cuda_status(pkv::launch_prefill_bf16(p, st));
+}
+
+int paged_kv_append(const void* k_new, const void* v_new, const int32_t* cu_new,
+                    const int32_t* start_pos, const int32_t* block_table, int max_pages_per_seq,
+                    int num_seqs, int num_new, void* k_pages, void* v_pages, int num_pages,
+                    int page_size, int H_kv, int d, int dtype, void* stream) {
+  if (num_new < 0 || num_seqs < 1 || max_pages_per_seq < 1 || num_pages < 1 || H_kv < 1 ||
+      !pow2(page_size) || page_size < 16 || page_size > 256 ||
+      (dtype != PKV_BF16 && dtype != PKV_F32))
+    return PKV_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return PKV_ERR_UNSUPPORTED;
+  if (num_new == 0) return PKV_OK;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pages) || !aligned16(v_pages) ||
+      !aligned4(cu_new) || !aligned4(start_pos) || !aligned4(block_table))
+    return PKV_ERR_INVALID_ARG;
+  if ((long long)num_pages * page_size > (1LL << 31)) return PKV_ERR_UNSUPPORTED;
+  unsigned int* err = nullptr;
+  if (int r = error_word(&err)) return r;
+  pkv::AppendParams p{};
+  p.k_new = k_new, p.v_new = v_new, p.cu_new = cu_new, p.start_pos = start_pos;
+  p.block_table = block_table, p.k_pages = k_pages, p.v_pages = v_pages, p.err = err;
+  p.num_seqs = num_seqs, p.num_new = num_new, p.max_pages = max_pages_per_seq;
+  p.num_pages = num_pages, p.page_size = page_size, p.page_shift = log2i(page_size);
+  p.row_bytes = (size_t)H_kv * d * (dtype == PKV_BF16 ? 2 : 4);
+  return cuda_status(pkv::launch_append(p, static_cast<cudaStream_t>(stream)));
+}
+
+int paged_kv_copy_pages(void* k_pages, void* v_pages, const int32_t* src, const int32_t* dst,
+                        int n, int num_pages, int page_size, int H_kv, int d, int dtype,
+                        void* stream) {
+  if (n < 0 || num_pages < 1 || H_kv < 1 || !pow2(page_size) || page_size < 16 ||
+      page_size > 256 || (dtype != PKV_BF16 && dtype != PKV_F32))
+    return PKV_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return PKV_ERR_UNSUPPORTED;
+  if (n == 0) return PKV_OK;
+  if (!aligned16(k_pages) || !aligned16(v_pages) || !aligned4(src) || !aligned4(dst))
+    return PKV_ERR_INVALID_ARG;
+  unsigned int* err = nullptr;
+  if (int r = error_word(&err)) return r;
+  pkv::CopyPagesParams p{};
+  p.k_pages = k_pages, p.v_pages = v_pages, p.src = src, p.dst = dst, p.err = err;
+  p.n = n, p.num_pages = num_pages;
+  p.page_bytes = (size_t)page_size * H_kv * d * (dtype == PKV_BF16 ? 2 : 4);
+  return cuda_status(pkv::launch_copy_pages(p, static_cast<cudaStream_t>(stream)));
 }
 
 int pkv_last_device_error(void* stream, unsigned int* bits) {
