@@ -278,6 +278,7 @@ def run_gpu(args, rank, world, dist):
     e2e_ms = e0.elapsed_time(e1) / n_e2e
 
     append = measure_append(device, stream, peaks)
+    paged_study = measure_paged_study(dev, stream, peaks)
     total_ms, e2e_ms, pre_ms, dec_ms = reduce_max([total_ms, e2e_ms, pre_ms, dec_ms], dist,
                                                   device)
     ms_step = total_ms / args.steps
@@ -316,6 +317,7 @@ def run_gpu(args, rank, world, dist):
                 "note": "pinned host Q/K/V, q, block_table, seq_lens in and O, out back every "
                         "step; the KV page pool is resident device state"},
         "append": append,
+        "paged_vs_contiguous": paged_study,
         "gpu_launches": args.steps * meta["launches_per_step"],
         "clocks": clocks,
     }
@@ -346,6 +348,74 @@ def append_setup(device, seqs=64, tokens=512, page_size=16, H_kv=32, d=128):
                           num_pages, page_size, H_kv, d, B.PKV_BF16, stream)
     moved = 2 * 2 * rows * H_kv * d * 2           # read K,V rows + write them
     return run, moved, f"{seqs} seqs x {tokens} new tokens, H_kv={H_kv} d={d} bf16, page 16"
+
+
+def _to_pages(K, page_size, gen):
+    """[B, H, N, d] -> ([B*N/ps (+slack) pages, ps, H, d], table [B, N/ps]) over shuffled pages."""
+    import torch
+    Bn, H, N, d = K.shape
+    per = N // page_size
+    num_pages = Bn * per
+    perm = torch.randperm(num_pages, generator=gen).to(torch.int32)
+    table = perm.view(Bn, per)
+    pages = torch.empty(num_pages, page_size, H, d, dtype=K.dtype, device=K.device)
+    src = K.permute(0, 2, 1, 3).reshape(Bn * per, page_size, H, d)    # logical pages in order
+    pages[perm.to(K.device).long()] = src
+    return pages, table.to(K.device)
+
+
+def measure_paged_study(dev, stream, peaks, iters=20):
+    """The step's prefill with K/V read through shuffled page tables (16 and
+    256 tokens per page) against the contiguous kernel, and the last 512-query
+    chunk of each prompt (chunked prefill, bottom-right causal mask)."""
+    import torch
+
+    from paged_kv_cache_exact_b200 import accounting, api
+    Q, K, V = dev["Q"], dev["K"], dev["V"]
+    Bn, H, N, d = Q.shape
+    scale = d ** -0.5
+    gen = torch.Generator().manual_seed(1098)
+    lens = torch.full((Bn,), N, dtype=torch.int32, device=Q.device)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(iters):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / iters
+
+    O = torch.empty_like(Q)
+    flops = accounting.prefill_flops(Bn, H, N, N, d, True)
+    out = {"workload": f"prefill B={Bn} H={H} N={N} d={d} causal"}
+    out["contiguous_ms"] = timed(lambda: api.prefill(Q, K, V, True, scale, out=O, stream=stream))
+    for ps in (256, 16):
+        kp, tb = _to_pages(K, ps, gen)
+        vp = torch.empty_like(kp)                  # V follows K's table
+        per = N // ps
+        vsrc = V.permute(0, 2, 1, 3).reshape(Bn * per, ps, H, d)
+        vp[tb.reshape(-1).long()] = vsrc
+        ms = timed(lambda: api.paged(Q, kp, vp, tb, lens, ps, True, scale, max_seq_len=N,
+                                     out=O, stream=stream))
+        out[f"paged_ps{ps}_ms"] = ms
+        out[f"paged_ps{ps}_vs_contiguous"] = out["contiguous_ms"] / ms
+        if ps == 256:
+            qc = Q[:, :, N - 512:].contiguous()
+            oc = torch.empty_like(qc)
+            cms = timed(lambda: api.paged(qc, kp, vp, tb, lens, ps, True, scale, max_seq_len=N,
+                                          out=oc, stream=stream))
+            cfl = accounting.prefill_flops(Bn, H, 512, N, d, True)
+            out["chunked_prefill"] = {"workload": f"last 512 queries of each of {Bn} prompts of "
+                                                  f"{N} tokens, H={H}, page 256",
+                                      "ms": cms, "tflops": cfl / (cms / 1e3) / 1e12,
+                                      "frac": cfl / (cms / 1e3) / 1e12 / peaks["bf16_tflops"]}
+        del kp, vp
+    out["contiguous_tflops"] = flops / (out["contiguous_ms"] / 1e3) / 1e12
+    return out
 
 
 def measure_append(device, stream, peaks, iters=50):

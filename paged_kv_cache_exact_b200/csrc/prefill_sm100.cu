@@ -226,29 +226,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       int last_k = -1, last_v = -1;                  // last tile whose K / V load was issued
       const int rows_per_box = kPaged ? min(p.page_size, BN) : BN;
       const int n_valid_pages = kPaged ? (g.kv_len + p.page_size - 1) >> p.page_shift : 0;
-      // Token row of box i of tile j in the page pool (paged) -- ids outside
-      // the pool are flagged and replaced by page 0, so nothing outside it is read.
-      auto box_row = [&](int k0, int i) -> int {
-        const int t = k0 + i * rows_per_box;
-        int phys = p.block_table[(size_t)g.b * p.max_pages + (t >> p.page_shift)];
-        if (phys < 0 || phys >= p.num_pages) {
-          flag_error(p.err, PKV_DEVERR_BAD_PAGE);
-          phys = 0;
-        }
-        return phys * p.page_size + (t & (p.page_size - 1));
-      };
-      auto load_tile = [&](const CUtensorMap* tm, uint32_t smem_tile, uint32_t full_bar, int k0,
-                           int nbox) {
-        for (int c = 0; c < 2; ++c) {
-          const uint32_t dst = smem_tile + c * kHalfBytes;
-          if (kPaged) {
-            for (int i = 0; i < nbox; ++i)
-              tma_load_3d(dst + i * rows_per_box * 128, tm, c * 64, g.kvh, box_row(k0, i), full_bar);
-          } else {
-            tma_load_3d(dst, tm, c * 64, k0, g.b * p.H_kv + g.kvh, full_bar);
-          }
-        }
-      };
+      // Paged tiles: all table entries of a tile are loaded together, once,
+      // before any of its TMA loads (the loads are independent of one another
+      // and hit L1 after the first tile), and serve both K and V.
+      constexpr int kMaxBoxes = BN / 16;
+      const int32_t* trow = p.block_table + (size_t)g.b * p.max_pages;
       bool ok = true;
       for (int j = 0; j < n && ok; ++j) {
         const int st = j % kStages;
@@ -257,15 +239,61 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // boxes of this tile that hold tokens of the sequence (never past its last page)
         const int nbox = kPaged ? min(BN / rows_per_box, n_valid_pages - (k0 >> p.page_shift)) : 1;
         const uint32_t bytes = kPaged ? nbox * rows_per_box * 256 : kTileBytes;
+        int rows[kMaxBoxes];
+        if (kPaged && rows_per_box == BN) {
+          // one box per tile (pages of >= 128 tokens)
+          int phys = trow[k0 >> p.page_shift];
+          if (phys < 0 || phys >= p.num_pages) {
+            flag_error(p.err, PKV_DEVERR_BAD_PAGE);
+            phys = 0;
+          }
+          rows[0] = phys * p.page_size + (k0 & (p.page_size - 1));
+        } else if (kPaged) {
+#pragma unroll
+          for (int i = 0; i < kMaxBoxes; ++i)
+            rows[i] = i < nbox ? trow[(k0 + i * rows_per_box) >> p.page_shift] : 0;
+#pragma unroll
+          for (int i = 0; i < kMaxBoxes; ++i) {
+            if (rows[i] < 0 || rows[i] >= p.num_pages) {    // never read outside the pool
+              flag_error(p.err, PKV_DEVERR_BAD_PAGE);
+              rows[i] = 0;
+            }
+            rows[i] = rows[i] * p.page_size + ((k0 + i * rows_per_box) & (p.page_size - 1));
+          }
+        }
         ok = wait(kBarKEmpty + st, ph ^ 1);
         if (!ok) break;
         mbar_arrive_expect_tx(bar(kBarKFull + st), bytes);
-        load_tile(&tmK, sbase + kOffK + st * kTileBytes, bar(kBarKFull + st), k0, nbox);
+        for (int c = 0; c < 2; ++c) {
+          const uint32_t dst = sbase + kOffK + st * kTileBytes + c * kHalfBytes;
+          if (kPaged && rows_per_box == BN) {
+            tma_load_3d(dst, &tmK, c * 64, g.kvh, rows[0], bar(kBarKFull + st));
+          } else if (kPaged) {
+#pragma unroll
+            for (int i = 0; i < kMaxBoxes; ++i)
+              if (i < nbox)
+                tma_load_3d(dst + i * rows_per_box * 128, &tmK, c * 64, g.kvh, rows[i], bar(kBarKFull + st));
+          } else {
+            tma_load_3d(dst, &tmK, c * 64, k0, g.b * p.H_kv + g.kvh, bar(kBarKFull + st));
+          }
+        }
         last_k = j;
         ok = wait(kBarVEmpty + st, ph ^ 1);
         if (!ok) break;
         mbar_arrive_expect_tx(bar(kBarVFull + st), bytes);
-        load_tile(&tmV, sbase + kOffV + st * kTileBytes, bar(kBarVFull + st), k0, nbox);
+        for (int c = 0; c < 2; ++c) {
+          const uint32_t dst = sbase + kOffV + st * kTileBytes + c * kHalfBytes;
+          if (kPaged && rows_per_box == BN) {
+            tma_load_3d(dst, &tmV, c * 64, g.kvh, rows[0], bar(kBarVFull + st));
+          } else if (kPaged) {
+#pragma unroll
+            for (int i = 0; i < kMaxBoxes; ++i)
+              if (i < nbox)
+                tma_load_3d(dst + i * rows_per_box * 128, &tmV, c * 64, g.kvh, rows[i], bar(kBarVFull + st));
+          } else {
+            tma_load_3d(dst, &tmV, c * 64, k0, g.b * p.H_kv + g.kvh, bar(kBarVFull + st));
+          }
+        }
         last_v = j;
       }
       if (!ok) {

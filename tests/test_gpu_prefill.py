@@ -132,3 +132,16 @@ def test_long_paged_prefill_workload_sampled_rows():
     want = paged_ref_per_head(w, rows=rows)
     check_close(got[:, :, rows], want, "workload 5")
     _status_ok()
+
+
+@pytest.mark.slow
+def test_chunked_prefill_full_size_sampled_rows():
+    """The last 512-query chunk of four 4096-token prompts (bottom-right causal:
+    query i sees keys <= i + 3584), 32 heads, pages of 256: every head on 64
+    sampled rows, including the first and last of the chunk."""
+    w = make_paged(81, [4096] * 4, H=32, d=128, page_size=256, q_len=512, decoys=4)
+    got = _paged(w)
+    rows = np.array(sorted({0, 1, 127, 128, 255, 256, 510, 511} |
+                           set(np.random.default_rng(81).integers(0, 512, 56).tolist())))
+    check_close(got[:, :, rows], paged_ref_per_head(w, rows=rows), "chunked prefill")
+    _status_ok()
