@@ -548,6 +548,8 @@ PROFILE_CASES = {
     "decode16": "paged decode, 16 seqs x 32 heads, seq_lens U[512,8192], page_size 16 "
                 "(the step's decode distribution, a quarter of the sequences)",
     "append": "paged KV append, 64 seqs x 512 new tokens, H_kv=32 d=128 bf16, page 16",
+    "decode-gqa": "paged decode with grouped heads, 64 seqs x 64 query heads over 8 kv heads, "
+                  "seq_lens U[512,8192], page_size 16",
 }
 
 
@@ -571,17 +573,22 @@ def run_profile(args):
         O = torch.empty_like(Q)
         fn = lambda: api.prefill(Q, K, V, True, w.scale, out=O)
     else:
-        w = workload(5) if args.profile == "paged-prefill" else \
-            make_paged(1003, (512, 8192, 16), 32, 128, 16, q_len=1, decoys=16)
+        if args.profile == "paged-prefill":
+            w = workload(5)
+        elif args.profile == "decode-gqa":
+            w = make_paged(2003, (512, 8192, 64), 64, 128, 16, q_len=1, H_kv=8, decoys=64)
+        else:
+            w = make_paged(1003, (512, 8192, 16), 32, 128, 16, q_len=1, decoys=16)
         t = [x.to(dev) for x in (w.q, w.k_pages, w.v_pages, w.block_table, w.seq_lens)]
         O = torch.empty_like(t[0])
-        ws = api.workspace_for(w.num_seqs, 32, 128, w.max_seq_len, w.page_size, dev)
+        ws = api.workspace_for(w.num_seqs, w.q.shape[1], 128, w.max_seq_len, w.page_size, dev)
         fn = lambda: api.paged(*t, w.page_size, True, w.scale, max_seq_len=w.max_seq_len,
                                out=O, workspace=ws)
     for _ in range(args.steps):
         fn()
     torch.cuda.synchronize(dev)
-    units = int(w.seq_lens.sum()) * 32 if args.profile == "decode16" else None
+    units = (int(w.seq_lens.sum()) * w.k_pages.shape[2]
+             if args.profile in ("decode16", "decode-gqa") else None)
     print(json.dumps({"profile": args.profile, "case": PROFILE_CASES[args.profile],
                       "iterations": args.steps, "decode_units": units}))
 

@@ -23,6 +23,14 @@
 
 namespace pkv {
 namespace {
+PKV_DEVINLINE uint32_t sm100_smem_addr(const void* ptr) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(ptr));
+}
+}  // namespace
+}  // namespace pkv
+
+namespace pkv {
+namespace {
 
 constexpr int D = 128;
 constexpr int kThreads = 128;           // 4 warps = 8 half-warps
@@ -232,6 +240,292 @@ __global__ void __launch_bounds__(D) combine_kernel(const DecodeParams p) {
   p.out[sh * D + tid] = __float2bfloat16_rn(s_L > 0.f ? o / s_L : 0.f);
 }
 
+
+// ---------------------------------------------------------------------------
+// Grouped-query decode (H > H_kv): one CTA per (split, kv head, sequence,
+// group of up to 16 query heads).  Every K/V row of the split is read from
+// HBM once, into shared memory, and serves all query heads that share the kv
+// head ("Flash Attention: Fast, Memory-Efficient Attention for LLMs", section
+// "Attention Variants: MHA, GQA, MQA").  With 2..16 query rows per kv head the
+// scores and the PV product are small matrix products, done on the tensor
+// cores with mma.sync m16n8k16 (bf16 in, f32 accumulate): M = 16 query heads
+// (padded), N = 8 tokens (QK^T) or 8 head dims (PV), K = 16.  Each of the 4
+// warps streams its own 16-token chunks through a 2-stage cp.async ring
+// (XOR-swizzled rows, so ldmatrix reads are conflict-free), keeps a running
+// (max, sum, O) per query head, and the warps and splits are merged with the
+// same log-sum-exp algebra as the per-head kernel.
+// ---------------------------------------------------------------------------
+constexpr int kGqaWarps = 4;
+constexpr int kGqaThreads = kGqaWarps * 32;
+constexpr int kChunk = 16;                          // tokens per warp step
+constexpr int kRowBytes = D * 2;                    // 256 B per token row
+constexpr int kStageBytes = kChunk * kRowBytes;     // 4 KB per matrix per stage
+#ifndef PKV_GQA_STAGES
+#define PKV_GQA_STAGES 2
+#endif
+constexpr int kGqaStages = PKV_GQA_STAGES;          // cp.async ring depth per warp
+#ifndef PKV_GQA_CTAS_PER_SM
+#define PKV_GQA_CTAS_PER_SM 8
+#endif
+constexpr int kGqaCtasPerSm = PKV_GQA_CTAS_PER_SM;  // split planning target
+constexpr int kWarpSmem = kGqaStages * 2 * kStageBytes;   // stages x (K, V)
+
+PKV_DEVINLINE void cp_async16(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+PKV_DEVINLINE void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+PKV_DEVINLINE void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+PKV_DEVINLINE void cp_async_wait_2() { asm volatile("cp.async.wait_group 2;" ::: "memory"); }
+PKV_DEVINLINE void cp_async_wait_0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+PKV_DEVINLINE void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+PKV_DEVINLINE void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+// d[16x8 f32] += a[16x16 bf16, row-major] * b[16x8 bf16, col-major]
+PKV_DEVINLINE void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                  uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// byte offset of 16-byte chunk c of token row r inside a stage (rows of 256 B)
+PKV_DEVINLINE uint32_t swz(int r, int c) { return r * kRowBytes + ((c ^ (r & 7)) << 4); }
+
+__global__ void __launch_bounds__(kGqaThreads)
+decode_gqa_kernel(const DecodeParams p) {
+  extern __shared__ __align__(128) uint8_t gsm[];
+  const int split = blockIdx.x, s = blockIdx.z;
+  const int group = p.H / p.H_kv;                    // query heads per kv head
+  const int n_hg = (group + 15) / 16;                // 16-head groups per kv head
+  const int kvh = blockIdx.y / n_hg;
+  const int h0 = kvh * group + (blockIdx.y % n_hg) * 16;   // first query head of this CTA
+  const int nh = min(16, kvh * group + group - h0);        // query heads in this CTA
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t4 = lane & 3;
+
+  int L = p.seq_lens[s];
+  const int cap = min(p.max_seq_len, p.max_pages * p.page_size);
+  if (L < 1 || L > cap) {
+    if (split == 0 && blockIdx.y == 0 && tid == 0) flag_error(p.err, PKV_DEVERR_BAD_LEN);
+    L = max(0, min(L, cap));
+  }
+  if (L <= 0) {
+    if (split == 0)
+      for (int i = tid; i < nh * D; i += kGqaThreads)
+        p.out[((size_t)s * p.H + h0 + i / D) * D + i % D] = __float2bfloat16_rn(0.f);
+    return;
+  }
+  const int t_begin = split * p.split_tokens;
+  if (t_begin >= L) return;
+  const int t_end = min(L, t_begin + p.split_tokens);
+  const int nsplit = (L + p.split_tokens - 1) / p.split_tokens;
+
+  // shared memory: per-warp K/V rings, then the split's page ids
+  int* s_pages = reinterpret_cast<int*>(gsm + kGqaWarps * kWarpSmem);
+  const int lp0 = t_begin >> p.page_shift;
+  const int lp1 = (t_end - 1) >> p.page_shift;
+  for (int i = tid; i <= lp1 - lp0; i += kGqaThreads) {
+    int phys = p.block_table[(size_t)s * p.max_pages + lp0 + i];
+    if (phys < 0 || phys >= p.num_pages) {
+      flag_error(p.err, PKV_DEVERR_BAD_PAGE);
+      phys = -1;
+    }
+    s_pages[i] = phys;
+  }
+
+  // Q as the A operand (rows = query heads, padded to 16; k = head dim),
+  // pre-rounded bf16 exactly as stored.
+  uint32_t qa[D / 16][4];
+  {
+    const __nv_bfloat16* qs = p.q + ((size_t)s * p.H + h0) * D;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const int c0 = 16 * kk + 2 * t4;
+      const uint32_t* r0 = reinterpret_cast<const uint32_t*>(qs + (size_t)g * D);
+      const uint32_t* r1 = reinterpret_cast<const uint32_t*>(qs + (size_t)(g + 8) * D);
+      qa[kk][0] = g < nh ? r0[c0 / 2] : 0u;
+      qa[kk][1] = g + 8 < nh ? r1[c0 / 2] : 0u;
+      qa[kk][2] = g < nh ? r0[(c0 + 8) / 2] : 0u;
+      qa[kk][3] = g + 8 < nh ? r1[(c0 + 8) / 2] : 0u;
+    }
+  }
+  __syncthreads();                                   // s_pages ready
+
+  const uint32_t wbase = sm100_smem_addr(gsm) + warp * kWarpSmem;
+  auto k_stage = [&](int stage) { return wbase + stage * 2 * kStageBytes; };
+  auto v_stage = [&](int stage) { return wbase + stage * 2 * kStageBytes + kStageBytes; };
+  const size_t row_stride = (size_t)p.H_kv * D;
+  const __nv_bfloat16* kbase = p.k_pages + (size_t)kvh * D;
+  const __nv_bfloat16* vbase = p.v_pages + (size_t)kvh * D;
+  const int pmask = p.page_size - 1;
+
+  // this lane's copies: token rows (lane / 16) + 2 i, 16-byte column chunk lane % 16
+  auto prefetch = [&](int chunk, int stage) {
+    const int cc = lane & 15;
+#pragma unroll
+    for (int i = 0; i < kChunk / 2; ++i) {
+      const int r = (lane >> 4) + 2 * i;
+      const int tok = t_begin + chunk * kChunk + r;
+      int phys = -1;
+      if (tok < t_end) phys = s_pages[(tok >> p.page_shift) - lp0];
+      const bool ok = phys >= 0;
+      const size_t row = ok ? (((size_t)phys << p.page_shift) + (tok & pmask)) : 0;
+      cp_async16(k_stage(stage) + swz(r, cc), kbase + row * row_stride + cc * 8, ok);
+      cp_async16(v_stage(stage) + swz(r, cc), vbase + row * row_stride + cc * 8, ok);
+    }
+  };
+
+  float o[D / 8][4];
+#pragma unroll
+  for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.f, l_hi = 0.f;   // rows g, g + 8
+
+  const int n_chunks = (t_end - t_begin + kChunk - 1) / kChunk;
+  // ring of kGqaStages chunks per warp: this warp's chunks are warp, warp + 4, ...
+#pragma unroll
+  for (int i = 0; i < kGqaStages - 1; ++i) {
+    if (warp + i * kGqaWarps < n_chunks) prefetch(warp + i * kGqaWarps, i);
+    cp_async_commit();
+  }
+  int st = 0;
+  for (int c = warp; c < n_chunks; c += kGqaWarps) {
+    const int ahead = c + (kGqaStages - 1) * kGqaWarps;
+    if (ahead < n_chunks) prefetch(ahead, (st + kGqaStages - 1) % kGqaStages);
+    cp_async_commit();
+    if (kGqaStages == 3)                             // this chunk's group is complete
+      cp_async_wait_2();
+    else
+      cp_async_wait_1();
+    __syncwarp();
+
+    // S = Q K^T for 16 tokens: two n-tiles of 8 tokens
+    float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const int mi = lane >> 3, ri = lane & 7;
+      uint32_t b[4];
+      ldsm_x4(k_stage(st) + swz(8 * (mi >> 1) + ri, 2 * kk + (mi & 1)), b);
+      mma_bf16_16816(sc[0], qa[kk], b[0], b[1]);
+      mma_bf16_16816(sc[1], qa[kk], b[2], b[3]);
+    }
+    // online softmax per query head (rows g and g + 8), base 2
+    const int tok0 = t_begin + c * kChunk;
+    float mx_lo = -INFINITY, mx_hi = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const bool valid = tok0 + 8 * nt + 2 * t4 + e < t_end;
+        sc[nt][e] = valid ? sc[nt][e] * p.scale_log2 : -INFINITY;
+        sc[nt][2 + e] = valid ? sc[nt][2 + e] * p.scale_log2 : -INFINITY;
+        mx_lo = fmaxf(mx_lo, sc[nt][e]);
+        mx_hi = fmaxf(mx_hi, sc[nt][2 + e]);
+      }
+    mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 1));
+    mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 2));
+    mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 1));
+    mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 2));
+    const float mn_lo = fmaxf(m_lo, mx_lo), mn_hi = fmaxf(m_hi, mx_hi);
+    const float a_lo = ex2(m_lo - mn_lo), a_hi = ex2(m_hi - mn_hi);   // -inf - x -> 0
+    const float sub_lo = mn_lo == -INFINITY ? 0.f : mn_lo;
+    const float sub_hi = mn_hi == -INFINITY ? 0.f : mn_hi;
+    m_lo = mn_lo;
+    m_hi = mn_hi;
+    float pr[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        pr[nt][e] = ex2(sc[nt][e] - sub_lo);
+        pr[nt][2 + e] = ex2(sc[nt][2 + e] - sub_hi);
+      }
+    l_lo = l_lo * a_lo + (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
+    l_hi = l_hi * a_hi + (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]);
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) {
+      o[i][0] *= a_lo;
+      o[i][1] *= a_lo;
+      o[i][2] *= a_hi;
+      o[i][3] *= a_hi;
+    }
+    // P as the A operand: k = the chunk's 16 tokens
+    uint32_t pa[4];
+    pa[0] = pack_bf16x2(pr[0][0], pr[0][1]);
+    pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
+    pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
+    pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
+    // O += P V: 16 n-tiles of 8 head dims
+#pragma unroll
+    for (int nd = 0; nd < D / 8; nd += 2) {
+      const int mi = lane >> 3, ri = lane & 7;
+      uint32_t b[4];
+      ldsm_x4_t(v_stage(st) + swz(8 * (mi & 1) + ri, nd + (mi >> 1)), b);
+      mma_bf16_16816(o[nd], pa, b[0], b[1]);
+      mma_bf16_16816(o[nd + 1], pa, b[2], b[3]);
+    }
+    __syncwarp();                                    // stage st may be refilled
+    st = (st + 1) % kGqaStages;
+  }
+  cp_async_wait_0();
+  l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 1);
+  l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 2);
+  l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 1);
+  l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 2);
+  __syncthreads();                                   // rings no longer read: reuse as merge buffers
+
+  // merge the warps: per warp, O [16][D] f32 and (m, l) [16]
+  float* s_o = reinterpret_cast<float*>(gsm);                       // [warps][16][D]
+  float* s_ml = s_o + kGqaWarps * 16 * D;                           // [warps][16][2]
+#pragma unroll
+  for (int nd = 0; nd < D / 8; ++nd) {
+    const int col = 8 * nd + 2 * t4;
+    s_o[(warp * 16 + g) * D + col] = o[nd][0];
+    s_o[(warp * 16 + g) * D + col + 1] = o[nd][1];
+    s_o[(warp * 16 + g + 8) * D + col] = o[nd][2];
+    s_o[(warp * 16 + g + 8) * D + col + 1] = o[nd][3];
+  }
+  if (t4 == 0) {
+    s_ml[(warp * 16 + g) * 2] = m_lo;
+    s_ml[(warp * 16 + g) * 2 + 1] = l_lo;
+    s_ml[(warp * 16 + g + 8) * 2] = m_hi;
+    s_ml[(warp * 16 + g + 8) * 2 + 1] = l_hi;
+  }
+  __syncthreads();
+  for (int i = tid; i < nh * D; i += kGqaThreads) {
+    const int r = i / D, col = i % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kGqaWarps; ++w) M = fmaxf(M, s_ml[(w * 16 + r) * 2]);
+    float acc = 0.f, lsum = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kGqaWarps; ++w) {
+        const float wt = ex2(s_ml[(w * 16 + r) * 2] - M);
+        acc = fmaf(wt, s_o[(w * 16 + r) * D + col], acc);
+        lsum = fmaf(wt, s_ml[(w * 16 + r) * 2 + 1], lsum);
+      }
+    }
+    const size_t sh = (size_t)s * p.H + h0 + r;
+    if (nsplit == 1) {
+      p.out[sh * D + col] = __float2bfloat16_rn(lsum > 0.f ? acc / lsum : 0.f);
+    } else {
+      p.ws_o[(sh * p.max_splits + split) * D + col] = acc;
+      if (col == 0) p.ws_ml[sh * p.max_splits + split] = make_float2(M, lsum);
+    }
+  }
+}
 }  // namespace
 
 void decode_plan(int num_seqs, int H, int max_seq_len, int page_size,
@@ -251,9 +545,44 @@ void decode_plan(int num_seqs, int H, int max_seq_len, int page_size,
 }
 
 cudaError_t launch_decode_bf16(const DecodeParams& p, cudaStream_t stream) {
-  dim3 grid(p.max_splits, p.H, p.num_seqs);
-  decode_split_kernel<4><<<grid, kThreads, 0, stream>>>(p);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e;
+  if (p.H > p.H_kv) {
+    // grouped heads: one CTA per (split, kv head, 16 query heads, sequence)
+    const int n_hg = (p.H / p.H_kv + 15) / 16;
+    const size_t smem = kGqaWarps * kWarpSmem + kMaxSplitPages * sizeof(int);
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+      e = cudaFuncSetAttribute(decode_gqa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem);
+      if (e != cudaSuccess) return e;
+      attr_set[dev] = true;
+    }
+    // Longer splits than the per-head plan (each CTA now serves up to 16 heads):
+    // double while there are still ~8 CTAs per SM.  Fewer splits use less of
+    // the caller's workspace, laid out with the same stride rule.
+    DecodeParams q = p;
+    const long long pairs = (long long)p.num_seqs * p.H_kv * n_hg;
+    while (q.split_tokens < 4096 && q.split_tokens * 2 <= kMaxSplitPages * q.page_size &&
+           pairs * ((p.max_seq_len + 2LL * q.split_tokens - 1) / (2LL * q.split_tokens)) >=
+               148LL * kGqaCtasPerSm)
+      q.split_tokens *= 2;
+    q.max_splits = (p.max_seq_len + q.split_tokens - 1) / q.split_tokens;
+    dim3 grid(q.max_splits, p.H_kv * n_hg, p.num_seqs);
+    decode_gqa_kernel<<<grid, kGqaThreads, smem, stream>>>(q);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (q.max_splits > 1) {
+      combine_kernel<<<dim3(p.H, p.num_seqs), D, 0, stream>>>(q);
+      e = cudaGetLastError();
+    }
+    return e;
+  } else {
+    dim3 grid(p.max_splits, p.H, p.num_seqs);
+    decode_split_kernel<4><<<grid, kThreads, 0, stream>>>(p);
+  }
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (p.max_splits > 1) {
     combine_kernel<<<dim3(p.H, p.num_seqs), D, 0, stream>>>(p);

@@ -132,3 +132,24 @@ def test_bad_page_id_is_flagged_not_faulted():
     assert st == B.PKV_ERR_BAD_TABLE and bits & B.PKV_DEVERR_BAD_PAGE
     # sequence 0 is untouched by the bad entry
     check_close(got[:1], paged_ref_per_head(w, seqs=[0]), "good sequence")
+
+
+@pytest.mark.parametrize("H,H_kv", [(8, 4), (16, 4), (32, 4), (16, 1), (64, 2)])
+@pytest.mark.parametrize("ps", [16, 256])
+def test_decode_grouped_heads(H, H_kv, ps):
+    """Query heads sharing a kv head (2, 4, 8, 16 and 32 per kv head; the last
+    spans two CTAs of 16), ragged lengths including 1 and page edges."""
+    w = make_paged(18 + H, [1, 17, 300, 4097, 2 * ps], H=H, H_kv=H_kv, d=128, page_size=ps,
+                   q_len=1, decoys=3)
+    check_close(_run(w), paged_ref_per_head(w), f"decode H={H} H_kv={H_kv} ps={ps}")
+    assert _device_status()[0] == 0
+
+
+@pytest.mark.slow
+def test_decode_grouped_full_size():
+    """64 sequences x 64 query heads over 8 kv heads (Llama-3-70B-like), lengths
+    U[512, 8192], pages of 16."""
+    w = make_paged(2003, (512, 8192, 64), 64, 128, 16, q_len=1, H_kv=8, decoys=64)
+    err, rel = check_close(_run(w), paged_ref_per_head(w), "decode gqa 64/8 full size")
+    assert _device_status()[0] == 0
+    print(f"gqa 64/8: max abs err {err:.3e}, max rel err {rel:.3e}")
