@@ -186,12 +186,12 @@ def build_step(device):
                                      max_pages=dec.block_table.shape[1])
     max_len = dec.max_seq_len
 
-    def prefill(stream):
-        api.prefill(dev["Q"], dev["K"], dev["V"], True, pre.scale, out=dev["O"], stream=stream)
+    def prefill(stream, d=dev):
+        api.prefill(d["Q"], d["K"], d["V"], True, pre.scale, out=d["O"], stream=stream)
 
-    def decode(stream):
-        api.paged(dev["q"], dev["k_pages"], dev["v_pages"], dev["table"], dev["lens"], 16, True,
-                  dec.scale, max_seq_len=max_len, out=dev["out"], workspace=dev["ws"],
+    def decode(stream, d=dev):
+        api.paged(d["q"], dev["k_pages"], dev["v_pages"], d["table"], d["lens"], 16, True,
+                  dec.scale, max_seq_len=max_len, out=d["out"], workspace=dev["ws"],
                   stream=stream)
 
     meta = {"inputs": (pre, dec), "prefill_flops": flops, "decode_bytes": dbytes, "sum_L": int(dec.seq_lens.sum()),
@@ -260,22 +260,48 @@ def run_gpu(args, rank, world, dist):
     if st != 0:
         raise RuntimeError(f"device error in the timed region: {bits:#x}")
 
-    # end to end: host buffers in, results out, every step
+    # End to end, every step: the step's inputs from pinned host memory, its
+    # results back to pinned host memory.  Steps are pipelined over two device
+    # buffer sets and three streams: the copy of step i+1's inputs and of step
+    # i-1's results overlap step i's kernels (a serving loop would do the same).
     n_e2e = max(3, min(args.steps, 20))
+    in_keys, out_keys = ("Q", "K", "V", "q", "table", "lens"), ("O", "out")
+    bufs = [dev, {k: torch.empty_like(dev[k]) for k in in_keys + out_keys}]
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev = {(name, b): torch.cuda.Event() for name in ("in", "comp", "out") for b in (0, 1)}
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(device)
     e0.record(stream)
-    for _ in range(n_e2e):
-        for k in ("Q", "K", "V", "q", "table", "lens"):
-            dev[k].copy_(host[k], non_blocking=True)
-        step()
-        host["O"].copy_(dev["O"], non_blocking=True)
-        host["out"].copy_(dev["out"], non_blocking=True)
+    s_in.wait_event(e0)
+    s_out.wait_event(e0)
+    for i in range(n_e2e):
+        b = i % 2
+        d = bufs[b]
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(ev[("comp", b)])        # step i-2 done reading these inputs
+            for k in in_keys:
+                d[k].copy_(host[k], non_blocking=True)
+            ev[("in", b)].record(s_in)
+        stream.wait_event(ev[("in", b)])
+        if i >= 2:
+            stream.wait_event(ev[("out", b)])           # step i-2's results copied out
+        prefill(stream, d)
+        decode(stream, d)
+        ev[("comp", b)].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev[("comp", b)])
+            for k in out_keys:
+                host[k].copy_(d[k], non_blocking=True)
+            ev[("out", b)].record(s_out)
+    stream.wait_event(ev[("out", (n_e2e - 1) % 2)])
+    stream.wait_event(ev[("in", (n_e2e - 1) % 2)])
     e1.record(stream)
     torch.cuda.synchronize(device)
     barrier()
     e2e_ms = e0.elapsed_time(e1) / n_e2e
+    del bufs[1]
 
     append = measure_append(device, stream, peaks)
     paged_study = measure_paged_study(dev, stream, peaks)
@@ -287,15 +313,22 @@ def run_gpu(args, rank, world, dist):
                                world)
     pre_tf = meta["prefill_flops"] / (pre_ms / 1e3) / 1e12
     dec_gbs = meta["decode_bytes"] / (dec_ms / 1e3) / 1e9
+    # The dominant kernel is timed inside a loop of back-to-back steps lasting
+    # about a second under the 1 kW power cap: its tensor peak is the measured
+    # sustained figure (the burst fraction is kept beside it).
     if pre_ms >= dec_ms:
         roof = {"kernel": "prefill_kernel", "bound": "tensor", "achieved": pre_tf,
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": pre_tf / peaks["bf16_tflops"],
-                "traffic": ncu_traffic("prefill_kernel", PREFILL_SRC, 1.0)}
+                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                "frac": pre_tf / peaks["bf16_tflops_sustained"],
+                "frac_of_burst_peak": pre_tf / peaks["bf16_tflops"],
+                "traffic": ncu_traffic("prefill_kernel", PREFILL_SRC, 1.0),
+                "peak_source": f"MEASURED_PEAKS.json bf16_tflops_sustained ({peak_src}); "
+                               f"kernel timed inside {total_ms / 1e3:.2f} s of back-to-back steps"}
     else:
         roof = {"kernel": "decode_split_kernel (+ combine)", "bound": "hbm", "achieved": dec_gbs,
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": dec_gbs / peaks["hbm_gbs"],
-                "traffic": ncu_traffic("decode_split_kernel", DECODE_SRC, meta["decode_units"])}
-    roof["peak_source"] = f"MEASURED_PEAKS.json ({peak_src}, burst)"
+                "traffic": ncu_traffic("decode_split_kernel", DECODE_SRC, meta["decode_units"]),
+                "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({peak_src})"}
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -315,7 +348,8 @@ def run_gpu(args, rank, world, dist):
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": meta["h2d"],
                 "d2h_bytes_per_step": meta["d2h"], "ms_per_step": e2e_ms,
                 "note": "pinned host Q/K/V, q, block_table, seq_lens in and O, out back every "
-                        "step; the KV page pool is resident device state"},
+                        "step, pipelined over 2 buffer sets and 3 streams; the KV page pool is "
+                        "resident device state"},
         "append": append,
         "paged_vs_contiguous": paged_study,
         "gpu_launches": args.steps * meta["launches_per_step"],
