@@ -305,6 +305,7 @@ def run_gpu(args, rank, world, dist):
 
     append = measure_append(device, stream, peaks)
     paged_study = measure_paged_study(dev, stream, peaks)
+    fp8 = measure_fp8(dev, stream, peaks)
     total_ms, e2e_ms, pre_ms, dec_ms = reduce_max([total_ms, e2e_ms, pre_ms, dec_ms], dist,
                                                   device)
     ms_step = total_ms / args.steps
@@ -352,6 +353,7 @@ def run_gpu(args, rank, world, dist):
                         "resident device state"},
         "append": append,
         "paged_vs_contiguous": paged_study,
+        "fp8_qk_prefill": fp8,
         "gpu_launches": args.steps * meta["launches_per_step"],
         "clocks": clocks,
     }
@@ -450,6 +452,38 @@ def measure_paged_study(dev, stream, peaks, iters=20):
         del kp, vp
     out["contiguous_tflops"] = flops / (out["contiguous_ms"] / 1e3) / 1e12
     return out
+
+
+def measure_fp8(dev, stream, peaks, iters=20):
+    """The step's prefill with e4m3 Q and K (per-tensor scales; S = QK^T on the
+    FP8 tensor-core path, PV in bf16)."""
+    import torch
+
+    from paged_kv_cache_exact_b200 import accounting
+    from paged_kv_cache_exact_b200 import binding as B
+    Q, K, V = dev["Q"], dev["K"], dev["V"]
+    Bn, H, N, d = Q.shape
+    qd = float(Q.float().abs().max()) / 448.0
+    kd = float(K.float().abs().max()) / 448.0
+    Q8 = (Q.float() / qd).to(torch.float8_e4m3fn).view(torch.uint8)
+    K8 = (K.float() / kd).to(torch.float8_e4m3fn).view(torch.uint8)
+    O = torch.empty_like(V)
+
+    def run():
+        B.attn_prefill_fp8qk(Q8, K8, V, O, Bn, H, N, d, True, d ** -0.5, qd, kd, stream)
+    for _ in range(3):
+        run()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(iters):
+        run()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / iters
+    tf = accounting.prefill_flops(Bn, H, N, N, d, True) / (ms / 1e3) / 1e12
+    return {"workload": f"causal prefill B={Bn} H={H} N={N} d={d}, e4m3 Q/K, bf16 V/O",
+            "ms": ms, "tflops": tf, "frac_of_bf16_peak": tf / peaks["bf16_tflops"]}
 
 
 def measure_append(device, stream, peaks, iters=50):

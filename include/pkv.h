@@ -97,6 +97,27 @@ PKV_API int attn_prefill(const void* Q, const void* K, const void* V, void* O,
                  int dtype, void* stream);
 
 /*
+ * attn_prefill_fp8qk - attention with e4m3 (FP8) Q and K, bf16 V and output.
+ *
+ * Defines: "Flash Attention: Fast, Memory-Efficient Attention for LLMs",
+ * section "Flash Attention 3" (FP8 tensor cores for the QK^T product).  What
+ * is computed, exactly as attn_prefill does it otherwise:
+ *
+ *     O = softmax((q_descale * Q8) (k_descale * K8)^T * scale) V
+ *
+ * where Q8, K8 hold e4m3 codes (1 sign, 4 exponent bits with bias 7, 3
+ * mantissa bits; no infinities) and the descales are the per-tensor factors
+ * the caller quantized with.  S = Q K^T runs on tcgen05 kind::f8f6f4; P and V
+ * stay bf16 for the PV product.
+ *
+ * Q8, K8 : device, [B, H, N, d] e4m3 bytes.   V, O : device, [B, H, N, d] bf16.
+ * d      : 128.  scale, q_descale, k_descale: finite and > 0.
+ */
+PKV_API int attn_prefill_fp8qk(const void* Q8, const void* K8, const void* V, void* O,
+                               int B, int H, int N, int d, int causal, float scale,
+                               float q_descale, float k_descale, void* stream);
+
+/*
  * paged_attn_workspace_size - bytes of scratch paged_attn needs.
  *
  * Decode (q_len == 1) splits each sequence's keys into fixed-size chunks that

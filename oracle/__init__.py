@@ -5,6 +5,7 @@ from .attention import (  # noqa: F401
     allowed_keys,
     attention_ref,
     bf16_bits_to_f64,
+    e4m3_bits_to_f64,
     gather_kv,
     lse_combine_ref,
     mha_ref,

@@ -66,6 +66,22 @@ def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
     return u.view(np.float32).astype(np.float64)
 
 
+def e4m3_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Decode FP8 e4m3 codes (uint8) to float64, exactly.
+
+    Bit 7 is the sign, bits 6..3 the exponent (bias 7), bits 2..0 the
+    mantissa.  Exponent 0 is subnormal (m/8 * 2^-6); exponent 15 with mantissa
+    7 is NaN; there are no infinities.
+    """
+    b = np.asarray(bits).view(np.uint8).astype(np.int64)
+    sign = np.where(b >> 7, -1.0, 1.0)
+    e = (b >> 3) & 0xF
+    m = b & 0x7
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    mag = np.where((e == 15) & (m == 7), np.nan, mag)
+    return sign * mag
+
+
 def to_f64(x: np.ndarray) -> np.ndarray:
     """float arrays are upcast; 16-bit integer arrays are read as bf16 bits."""
     x = np.asarray(x)

@@ -36,6 +36,8 @@ _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_
 
 _lib.attn_prefill.restype = _i
 _lib.attn_prefill.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _vp]
+_lib.attn_prefill_fp8qk.restype = _i
+_lib.attn_prefill_fp8qk.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _f, _f, _vp]
 _lib.paged_attn_workspace_size.restype = _sz
 _lib.paged_attn_workspace_size.argtypes = [_i, _i, _i, _i, _i]
 _lib.paged_attn.restype = _i
@@ -113,6 +115,13 @@ def pkv_status_string(status: int) -> str:
 def attn_prefill(Q, K, V, O, B, H, N, d, causal, scale, dtype, stream=None):
     _check("attn_prefill", _lib.attn_prefill(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), B, H, N, d,
                                              int(causal), float(scale), dtype, _stream(stream)))
+
+
+def attn_prefill_fp8qk(Q8, K8, V, O, B, H, N, d, causal, scale, q_descale, k_descale,
+                       stream=None):
+    _check("attn_prefill_fp8qk", _lib.attn_prefill_fp8qk(
+        _ptr(Q8), _ptr(K8), _ptr(V), _ptr(O), B, H, N, d, int(causal), float(scale),
+        float(q_descale), float(k_descale), _stream(stream)))
 
 
 def paged_attn_workspace_size(num_seqs, H, d, max_seq_len, page_size) -> int:

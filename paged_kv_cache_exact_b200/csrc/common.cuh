@@ -89,6 +89,7 @@ struct PrefillParams {
   int causal;
   float scale_log2;
   int head_group;   // (batch, head) pairs scheduled together (set by the launcher)
+  int fp8_qk;       // Q and K are e4m3 (contiguous only); V and O stay bf16
 };
 
 struct AppendParams {

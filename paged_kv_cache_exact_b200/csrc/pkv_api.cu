@@ -114,6 +114,26 @@ int attn_prefill(const void* Q, const void* K, const void* V, void* O, int B, in
   return PKV_ERR_INVALID_ARG;
 }
 
+int attn_prefill_fp8qk(const void* Q8, const void* K8, const void* V, void* O, int B, int H,
+                       int N, int d, int causal, float scale, float q_descale, float k_descale,
+                       void* stream) {
+  if (!aligned16(Q8) || !aligned16(K8) || !aligned16(V) || !aligned16(O)) return PKV_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1 || (causal != 0 && causal != 1) || !good_scale(scale) ||
+      !good_scale(q_descale) || !good_scale(k_descale))
+    return PKV_ERR_INVALID_ARG;
+  if (d != 128) return PKV_ERR_UNSUPPORTED;
+  if (B > 65535 || H > 65535) return PKV_ERR_UNSUPPORTED;
+  unsigned int* err = nullptr;
+  if (int r = error_word(&err)) return r;
+  pkv::PrefillParams p{};
+  p.Q = Q8, p.K = K8, p.V = V, p.O = O;
+  p.err = err;
+  p.B = B, p.H = H, p.H_kv = H, p.q_len = N, p.kv_len = N, p.d = d;
+  p.paged = 0, p.causal = causal, p.fp8_qk = 1;
+  p.scale_log2 = scale * q_descale * k_descale * pkv::kLog2e;
+  return cuda_status(pkv::launch_prefill_bf16(p, static_cast<cudaStream_t>(stream)));
+}
+
 size_t paged_attn_workspace_size(int num_seqs, int H, int d, int max_seq_len, int page_size) {
   if (num_seqs < 1 || H < 1 || d < 1 || max_seq_len < 1 || !pow2(page_size)) return 0;
   int split = 0, nsplit = 0;

@@ -113,6 +113,10 @@ constexpr uint32_t kColS = 0;      // + 128 * tile
 constexpr uint32_t kColO = 256;    // + 128 * tile
 
 constexpr uint32_t kIdescS = make_idesc_bf16(BM, BN, false);  // Q (K-major) x K (K-major)
+constexpr uint32_t kIdescS8 = make_idesc_e4m3(BM, BN);         // e4m3 Q x e4m3 K
+// e4m3 Q/K tiles: 128 rows of 128 one-byte elements, a single 128-byte-swizzled
+// column block (16 KB) at the start of the same 32 KB slots the bf16 tiles use.
+constexpr int kTileBytes8 = BM * D;
 constexpr uint32_t kIdescO = make_idesc_bf16(BM, D, true);    // P (TMEM) x V (MN-major)
 
 struct Geometry {
@@ -161,7 +165,7 @@ __device__ __forceinline__ Geometry cta_geometry(const PrefillParams& p) {
 }
 
 // ----------------------------------------------------------------------------
-template <bool kPaged>
+template <bool kPaged, bool kFp8QK>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
@@ -218,9 +222,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
       const int qc2 = g.b * p.H + g.h;
-      mbar_arrive_expect_tx(bar(kBarQ), kQTiles * kTileBytes);
+      mbar_arrive_expect_tx(bar(kBarQ), kQTiles * (kFp8QK ? kTileBytes8 : kTileBytes));
       for (int t = 0; t < kQTiles; ++t)
-        for (int c = 0; c < 2; ++c)
+        for (int c = 0; c < (kFp8QK ? 1 : 2); ++c)
           tma_load_3d(sbase + kOffQ + t * kTileBytes + c * kHalfBytes, &tmQ, c * 64,
                       g.q0 + t * BM, qc2, bar(kBarQ));
       int last_k = -1, last_v = -1;                  // last tile whose K / V load was issued
@@ -263,8 +267,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         ok = wait(kBarKEmpty + st, ph ^ 1);
         if (!ok) break;
-        mbar_arrive_expect_tx(bar(kBarKFull + st), bytes);
-        for (int c = 0; c < 2; ++c) {
+        mbar_arrive_expect_tx(bar(kBarKFull + st), kFp8QK ? kTileBytes8 : bytes);
+        for (int c = 0; c < (kFp8QK ? 1 : 2); ++c) {
           const uint32_t dst = sbase + kOffK + st * kTileBytes + c * kHalfBytes;
           if (kPaged && rows_per_box == BN) {
             tma_load_3d(dst, &tmK, c * 64, g.kvh, rows[0], bar(kBarKFull + st));
@@ -358,10 +362,16 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const uint64_t dq = t ? dq1 : dq0;
         const uint32_t tS = tmem + kColS + 128 * t;
         if (leader) {
+          if (kFp8QK) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t koff = ((kk / 4) * kHalfBytes + (kk % 4) * 32) >> 4;
-            mma_ss(tS, dq + koff, dk + koff, kIdescS, kk > 0);
+            for (int kk = 0; kk < D / 32; ++kk)     // K = 32 e4m3 (32 bytes) per MMA
+              mma_ss_f8(tS, dq + ((kk * 32) >> 4), dk + ((kk * 32) >> 4), kIdescS8, kk > 0);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t koff = ((kk / 4) * kHalfBytes + (kk % 4) * 32) >> 4;
+              mma_ss(tS, dq + koff, dk + koff, kIdescS, kk > 0);
+            }
           }
           mma_commit(bar(kBarSFull + t));
         }
@@ -618,22 +628,25 @@ EncodeFn get_encode() {
   return fn;
 }
 
-// 3-D bf16 map, 128-byte swizzle, box {64, box1, box2}; out-of-range reads fill zeros.
+// 3-D map, 128-byte swizzle, box {128 bytes of d, box1, box2} (64 bf16 or 128 e4m3);
+// out-of-range reads fill zeros.
 bool encode_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
-               uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box1, uint32_t box2) {
+               uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box1, uint32_t box2,
+               bool bytes = false) {
   EncodeFn enc = get_encode();
   if (!enc) return false;
   const cuuint64_t dims[3] = {d0, d1, d2};
   const cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
-  const cuuint32_t box[3] = {64, box1, box2};
+  const cuuint32_t box[3] = {bytes ? 128u : 64u, box1, box2};
   const cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+  return enc(m, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+             const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
 }
 
-template <bool kPaged>
+template <bool kPaged, bool kFp8QK>
 cudaError_t set_smem_attr() {
   static int done[64] = {};
   int dev = 0;
@@ -641,10 +654,10 @@ cudaError_t set_smem_attr() {
   if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
   // The in-kernel register split assumes this exact launch allocation.
   cudaFuncAttributes fa;
-  cudaError_t e = cudaFuncGetAttributes(&fa, prefill_kernel<kPaged>);
+  cudaError_t e = cudaFuncGetAttributes(&fa, prefill_kernel<kPaged, kFp8QK>);
   if (e != cudaSuccess) return e;
   if (fa.numRegs != kLaunchRegs) return cudaErrorNotSupported;
-  e = cudaFuncSetAttribute(prefill_kernel<kPaged>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(prefill_kernel<kPaged, kFp8QK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kSmemBytes);
   if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = 1;
   return e;
@@ -656,8 +669,11 @@ cudaError_t launch_prefill_bf16(const PrefillParams& p, cudaStream_t stream) {
   if (p.d != D) return cudaErrorNotSupported;
   CUtensorMap tq, tk, tv;
   const uint64_t row_bytes = D * 2;
+  const bool f8 = p.fp8_qk != 0;
+  if (f8 && p.paged) return cudaErrorNotSupported;
+  const uint64_t qk_row = f8 ? D : row_bytes;        // e4m3 Q/K rows are 128 bytes
   // Q: [B*H, q_len, d]
-  if (!encode_3d(&tq, p.Q, D, p.q_len, (uint64_t)p.B * p.H, row_bytes, row_bytes * p.q_len, BM, 1))
+  if (!encode_3d(&tq, p.Q, D, p.q_len, (uint64_t)p.B * p.H, qk_row, qk_row * p.q_len, BM, 1, f8))
     return cudaErrorInvalidValue;
   if (p.paged) {
     // pages [P, ps, H_kv, d] viewed as [P*ps tokens, H_kv, d]; one box = one page's rows.
@@ -668,7 +684,7 @@ cudaError_t launch_prefill_bf16(const PrefillParams& p, cudaStream_t stream) {
       return cudaErrorInvalidValue;
   } else {
     const uint64_t bhkv = (uint64_t)p.B * p.H_kv;
-    if (!encode_3d(&tk, p.K, D, p.kv_len, bhkv, row_bytes, row_bytes * p.kv_len, BN, 1) ||
+    if (!encode_3d(&tk, p.K, D, p.kv_len, bhkv, qk_row, qk_row * p.kv_len, BN, 1, f8) ||
         !encode_3d(&tv, p.V, D, p.kv_len, bhkv, row_bytes, row_bytes * p.kv_len, BN, 1))
       return cudaErrorInvalidValue;
   }
@@ -689,13 +705,17 @@ cudaError_t launch_prefill_bf16(const PrefillParams& p, cudaStream_t stream) {
   }
   cudaError_t e;
   if (p.paged) {
-    e = set_smem_attr<true>();
+    e = set_smem_attr<true, false>();
     if (e != cudaSuccess) return e;
-    prefill_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, q);
+    prefill_kernel<true, false><<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, q);
+  } else if (f8) {
+    e = set_smem_attr<false, true>();
+    if (e != cudaSuccess) return e;
+    prefill_kernel<false, true><<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, q);
   } else {
-    e = set_smem_attr<false>();
+    e = set_smem_attr<false, false>();
     if (e != cudaSuccess) return e;
-    prefill_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, q);
+    prefill_kernel<false, false><<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, q);
   }
   return cudaGetLastError();
 }

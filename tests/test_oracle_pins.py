@@ -360,3 +360,17 @@ def test_generator_poison_and_fixed_table():
                                      w.v_pages.view(torch.int16).numpy(), w.block_table.numpy(),
                                      w.seq_lens.numpy(), 256, True, w.scale)
     assert np.isfinite(got).all()
+
+
+def test_e4m3_decoding_all_codes():
+    """Every e4m3 code decodes as torch's float8_e4m3fn does (library special
+    case), plus values fixed by the format: 1.0, the largest finite 448, the
+    smallest subnormal 2^-9, and the two NaN codes."""
+    codes = np.arange(256, dtype=np.uint8)
+    got = oracle.e4m3_bits_to_f64(codes)
+    want = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(got), np.isnan(want))
+    ok = ~np.isnan(want)
+    assert np.array_equal(got[ok], want[ok])
+    assert got[0x38] == 1.0 and got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9
+    assert got[0xB8] == -1.0 and np.isnan(got[0x7F]) and np.isnan(got[0xFF])
