@@ -612,6 +612,8 @@ def run_reference(args):
 
 PROFILE_CASES = {
     "prefill": "causal prefill B=4 H=32 N=4096 d=128 (the step's prefill, 1 launch/iter)",
+    "prefill-fp8": "causal prefill B=4 H=32 N=4096 d=128, e4m3 Q/K with per-tensor scales, "
+                   "bf16 V/O",
     "paged-prefill": "paged causal prefill 1x32x32768x128, 128 shuffled pages of 256",
     "decode16": "paged decode, 16 seqs x 32 heads, seq_lens U[512,8192], page_size 16 "
                 "(the step's decode distribution, a quarter of the sequences)",
@@ -640,6 +642,17 @@ def run_profile(args):
         Q, K, V = w.Q.to(dev), w.K.to(dev), w.V.to(dev)
         O = torch.empty_like(Q)
         fn = lambda: api.prefill(Q, K, V, True, w.scale, out=O)
+    elif args.profile == "prefill-fp8":
+        from paged_kv_cache_exact_b200 import binding as B
+        w = workload(2)
+        Q, K, V = w.Q.to(dev), w.K.to(dev), w.V.to(dev)
+        qd = float(Q.float().abs().max()) / 448.0
+        kd = float(K.float().abs().max()) / 448.0
+        Q8 = (Q.float() / qd).to(torch.float8_e4m3fn).view(torch.uint8)
+        K8 = (K.float() / kd).to(torch.float8_e4m3fn).view(torch.uint8)
+        O = torch.empty_like(V)
+        Bn, H, N, d = Q.shape
+        fn = lambda: B.attn_prefill_fp8qk(Q8, K8, V, O, Bn, H, N, d, True, w.scale, qd, kd)
     else:
         if args.profile == "paged-prefill":
             w = workload(5)
