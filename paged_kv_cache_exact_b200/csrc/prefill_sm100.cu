@@ -204,7 +204,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     *abort_flag = 1;
     flag_error(p.err, PKV_DEVERR_TIMEOUT);
   };
+  // A phase that has already completed costs one try_wait; the abort flag (a
+  // shared-memory read) is consulted only once the caller has to wait.
   auto wait = [&](int b, uint32_t parity) -> bool {
+    if (mbar_try_wait(bar(b), parity)) return true;
     if (*abort_flag) return false;
     if (!mbar_wait_bounded(bar(b), parity, kWaitLimitNs)) {
       fail();
@@ -390,12 +393,16 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         __syncwarp();
       };
-      auto issue_pv = [&](int t, int j) -> bool {
+      // PV_t(j).  With want_k the next K tile is checked while the second half
+      // of P is still being written, so that PV's second half and S_t(j+1)
+      // issue back to back once P is complete.
+      auto issue_pv = [&](int t, int j, bool want_k = false) -> bool {
         if (kSplitP) {
           if (!wwait(kBarPHalf + t, j & 1)) return false;
           tc_fence_after();
           issue_pv_half(t, j, 0);
         }
+        if (want_k && !wwait(kBarKFull + (j + 1) % kStages, ((j + 1) / kStages) & 1)) return false;
         if (!wwait(kBarPFull + t, j & 1)) return false;
         tc_fence_after();
         if (!kSplitP) issue_pv_half(t, j, 0);
@@ -421,11 +428,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           ok = wwait(kBarVFixed, 0);
         else
           ok = wwait(kBarVFull + st, (j / kStages) & 1);
-        ok = ok && issue_pv(0, j);
+        ok = ok && issue_pv(0, j, j + 1 < n);
         if (!ok) break;
         if (j + 1 < n) {
-          ok = wwait(kBarKFull + (j + 1) % kStages, ((j + 1) / kStages) & 1);
-          if (!ok) break;
           tc_fence_after();
           issue_s(0, j + 1);
         }
