@@ -61,6 +61,28 @@ def test_dense_large_scores_no_overflow():
     check_close(got, want, "dense large scores")
 
 
+@pytest.mark.parametrize("growth", [7.5, 12.0, 40.0])
+@pytest.mark.parametrize("causal", [True, False])
+def test_running_max_staircase(growth, causal):
+    """Key scores that climb by `growth` (log2 units) per 128-key tile: at 12
+    and 40 every tile moves the row max past the 2^8 rescale threshold, at 7.5
+    none does, and the exponentials reach ~2^7.5 without a rescale."""
+    N, d, scale = 1000, 128, 0.088
+    g = torch.Generator().manual_seed(77)
+    log2e = 1.4426950408889634
+    c = torch.arange(N, dtype=torch.float64) * growth / 128.0 / (d * scale * log2e)
+    K = (c[:, None] * torch.ones(1, d, dtype=torch.float64)).to(torch.bfloat16)
+    K = K.expand(2, N, d).reshape(1, 2, N, d).contiguous()
+    Q = (1.0 + 0.05 * torch.randn(1, 2, N, d, generator=g)).to(torch.bfloat16)
+    V = torch.randn(1, 2, N, d, generator=g).to(torch.bfloat16)
+    from paged_kv_cache_exact_b200 import api
+    got = api.prefill(Q.cuda(), K.cuda(), V.cuda(), causal, scale)
+    torch.cuda.synchronize()
+    want = oracle.mha_ref(f64(Q), f64(K), f64(V), causal, scale)
+    check_close(got.cpu(), want, f"staircase growth={growth} causal={causal}")
+    _status_ok()
+
+
 @pytest.mark.slow
 def test_causal_prefill_workload_sampled_rows():
     """4 x 32 x 4096 x 128 causal: every head on 40 rows spanning tile edges,
