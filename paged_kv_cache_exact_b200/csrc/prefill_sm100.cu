@@ -220,23 +220,31 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer --
-    if (lane == 0 && n > 0) {
-      prefetch_tmap(&tmQ);
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
-      const int qc2 = g.b * p.H + g.h;
-      mbar_arrive_expect_tx(bar(kBarQ), kQTiles * (kFp8QK ? kTileBytes8 : kTileBytes));
-      for (int t = 0; t < kQTiles; ++t)
-        for (int c = 0; c < (kFp8QK ? 1 : 2); ++c)
-          tma_load_3d(sbase + kOffQ + t * kTileBytes + c * kHalfBytes, &tmQ, c * 64,
-                      g.q0 + t * BM, qc2, bar(kBarQ));
+    // The warp runs the loop converged.  Contiguous tiles and pages of >= 128
+    // tokens take one TMA box per 64-column block, issued by lane 0; shorter
+    // pages take one box per page per block, and lane i resolves page i of the
+    // tile and issues its boxes, so the boxes of a tile are issued in parallel
+    // (one thread issuing 16 of them per K or V tile could not keep ahead of
+    // the tensor core).  Each table entry is read once and serves K and V.
+    if (n > 0) {
+      if (lane == 0) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+        const int qc2 = g.b * p.H + g.h;
+        mbar_arrive_expect_tx(bar(kBarQ), kQTiles * (kFp8QK ? kTileBytes8 : kTileBytes));
+        for (int t = 0; t < kQTiles; ++t)
+          for (int c = 0; c < (kFp8QK ? 1 : 2); ++c)
+            tma_load_3d(sbase + kOffQ + t * kTileBytes + c * kHalfBytes, &tmQ, c * 64,
+                        g.q0 + t * BM, qc2, bar(kBarQ));
+      }
+      auto wwait = [&](int b, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu, wait(b, parity));
+      };
       int last_k = -1, last_v = -1;                  // last tile whose K / V load was issued
       const int rows_per_box = kPaged ? min(p.page_size, BN) : BN;
+      const bool box_per_page = kPaged && rows_per_box < BN;
       const int n_valid_pages = kPaged ? (g.kv_len + p.page_size - 1) >> p.page_shift : 0;
-      // Paged tiles: all table entries of a tile are loaded together, once,
-      // before any of its TMA loads (the loads are independent of one another
-      // and hit L1 after the first tile), and serve both K and V.
-      constexpr int kMaxBoxes = BN / 16;
       const int32_t* trow = p.block_table + (size_t)g.b * p.max_pages;
       bool ok = true;
       for (int j = 0; j < n && ok; ++j) {
@@ -246,64 +254,48 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // boxes of this tile that hold tokens of the sequence (never past its last page)
         const int nbox = kPaged ? min(BN / rows_per_box, n_valid_pages - (k0 >> p.page_shift)) : 1;
         const uint32_t bytes = kPaged ? nbox * rows_per_box * 256 : kTileBytes;
-        int rows[kMaxBoxes];
-        if (kPaged && rows_per_box == BN) {
-          // one box per tile (pages of >= 128 tokens)
-          int phys = trow[k0 >> p.page_shift];
-          if (phys < 0 || phys >= p.num_pages) {
+        // this lane's box: first token row of its page slice in the pool
+        const int mine = box_per_page ? lane : 0;
+        int row = 0;
+        if (kPaged && mine < nbox) {
+          int phys = trow[(k0 + mine * rows_per_box) >> p.page_shift];
+          if (phys < 0 || phys >= p.num_pages) {     // never read outside the pool
             flag_error(p.err, PKV_DEVERR_BAD_PAGE);
             phys = 0;
           }
-          rows[0] = phys * p.page_size + (k0 & (p.page_size - 1));
-        } else if (kPaged) {
-#pragma unroll
-          for (int i = 0; i < kMaxBoxes; ++i)
-            rows[i] = i < nbox ? trow[(k0 + i * rows_per_box) >> p.page_shift] : 0;
-#pragma unroll
-          for (int i = 0; i < kMaxBoxes; ++i) {
-            if (rows[i] < 0 || rows[i] >= p.num_pages) {    // never read outside the pool
-              flag_error(p.err, PKV_DEVERR_BAD_PAGE);
-              rows[i] = 0;
-            }
-            rows[i] = rows[i] * p.page_size + ((k0 + i * rows_per_box) & (p.page_size - 1));
-          }
+          row = phys * p.page_size + ((k0 + mine * rows_per_box) & (p.page_size - 1));
         }
-        ok = wait(kBarKEmpty + st, ph ^ 1);
+        const bool issues = box_per_page ? lane < nbox : lane == 0;
+        ok = wwait(kBarKEmpty + st, ph ^ 1);
         if (!ok) break;
-        mbar_arrive_expect_tx(bar(kBarKFull + st), kFp8QK ? kTileBytes8 : bytes);
-        for (int c = 0; c < (kFp8QK ? 1 : 2); ++c) {
-          const uint32_t dst = sbase + kOffK + st * kTileBytes + c * kHalfBytes;
-          if (kPaged && rows_per_box == BN) {
-            tma_load_3d(dst, &tmK, c * 64, g.kvh, rows[0], bar(kBarKFull + st));
-          } else if (kPaged) {
-#pragma unroll
-            for (int i = 0; i < kMaxBoxes; ++i)
-              if (i < nbox)
-                tma_load_3d(dst + i * rows_per_box * 128, &tmK, c * 64, g.kvh, rows[i], bar(kBarKFull + st));
-          } else {
-            tma_load_3d(dst, &tmK, c * 64, k0, g.b * p.H_kv + g.kvh, bar(kBarKFull + st));
+        if (lane == 0) mbar_arrive_expect_tx(bar(kBarKFull + st), kFp8QK ? kTileBytes8 : bytes);
+        __syncwarp();
+        if (issues) {
+          for (int c = 0; c < (kFp8QK ? 1 : 2); ++c) {
+            const uint32_t dst = sbase + kOffK + st * kTileBytes + c * kHalfBytes;
+            if (kPaged)
+              tma_load_3d(dst + mine * rows_per_box * 128, &tmK, c * 64, g.kvh, row, bar(kBarKFull + st));
+            else
+              tma_load_3d(dst, &tmK, c * 64, k0, g.b * p.H_kv + g.kvh, bar(kBarKFull + st));
           }
         }
         last_k = j;
-        ok = wait(kBarVEmpty + st, ph ^ 1);
+        ok = wwait(kBarVEmpty + st, ph ^ 1);
         if (!ok) break;
-        mbar_arrive_expect_tx(bar(kBarVFull + st), bytes);
-        for (int c = 0; c < 2; ++c) {
-          const uint32_t dst = sbase + kOffV + st * kTileBytes + c * kHalfBytes;
-          if (kPaged && rows_per_box == BN) {
-            tma_load_3d(dst, &tmV, c * 64, g.kvh, rows[0], bar(kBarVFull + st));
-          } else if (kPaged) {
-#pragma unroll
-            for (int i = 0; i < kMaxBoxes; ++i)
-              if (i < nbox)
-                tma_load_3d(dst + i * rows_per_box * 128, &tmV, c * 64, g.kvh, rows[i], bar(kBarVFull + st));
-          } else {
-            tma_load_3d(dst, &tmV, c * 64, k0, g.b * p.H_kv + g.kvh, bar(kBarVFull + st));
+        if (lane == 0) mbar_arrive_expect_tx(bar(kBarVFull + st), bytes);
+        __syncwarp();
+        if (issues) {
+          for (int c = 0; c < 2; ++c) {
+            const uint32_t dst = sbase + kOffV + st * kTileBytes + c * kHalfBytes;
+            if (kPaged)
+              tma_load_3d(dst + mine * rows_per_box * 128, &tmV, c * 64, g.kvh, row, bar(kBarVFull + st));
+            else
+              tma_load_3d(dst, &tmV, c * 64, k0, g.b * p.H_kv + g.kvh, bar(kBarVFull + st));
           }
         }
         last_v = j;
       }
-      if (!ok) {
+      if (!ok && lane == 0) {
         // Drain loads already in flight before the CTA's shared memory goes away.
         for (int jj = max(0, last_k - 1); jj <= last_k; ++jj)
           mbar_wait_bounded(bar(kBarKFull + jj % kStages), (jj / kStages) & 1, kWaitLimitNs);
