@@ -233,6 +233,12 @@ PKV_API int paged_decode_noalloc(const void* q, const void* k_pages, const void*
  * A row whose page id is outside [0, num_pages) or whose position is past the
  * table is skipped and flagged (PKV_DEVERR_BAD_PAGE / PKV_DEVERR_BAD_LEN).
  * Rows must not target the same slot twice in one call.
+ * Returns PKV_OK without reading any pointer or launching when num_new == 0;
+ * PKV_ERR_INVALID_ARG for a negative num_new, num_seqs, max_pages_per_seq,
+ * num_pages or H_kv below 1, a page_size that is not a power of two in
+ * [16, 256], an unknown dtype, or a null or misaligned pointer (16 bytes for
+ * row data, 4 for the int32 arrays); PKV_ERR_UNSUPPORTED for d other than 64
+ * or 128, or a pool of more than 2^31 token rows.
  */
 PKV_API int paged_kv_append(const void* k_new, const void* v_new, const int32_t* cu_new,
                             const int32_t* start_pos, const int32_t* block_table,
@@ -248,6 +254,11 @@ PKV_API int paged_kv_append(const void* k_new, const void* v_new, const int32_t*
  * works": sequences share prefix blocks and copy only when they diverge).
  * src, dst : device int32 [n]; ids in [0, num_pages) (others are skipped and
  *            flagged); a dst must not also be a src in the same call.
+ * Returns PKV_OK without reading any pointer or launching when n == 0;
+ * PKV_ERR_INVALID_ARG for a negative n, num_pages or H_kv below 1, a page_size
+ * that is not a power of two in [16, 256], an unknown dtype, or a null or
+ * misaligned pointer (16 bytes for the pools, 4 for src and dst);
+ * PKV_ERR_UNSUPPORTED for d other than 64 or 128.
  */
 PKV_API int paged_kv_copy_pages(void* k_pages, void* v_pages, const int32_t* src,
                                 const int32_t* dst, int n, int num_pages, int page_size,

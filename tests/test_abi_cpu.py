@@ -124,3 +124,74 @@ def test_no_alloc_decode_rejects_plans_beyond_its_scratch():
     st = B.raw_status("paged_decode_noalloc", FAKE, FAKE, FAKE, FAKE, FAKE, ps, 4, H, H, 64,
                       64, L // ps, L, ctypes.c_float(0.1), FAKE, None)
     assert st == B.PKV_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(Q8=None), B.PKV_ERR_INVALID_ARG),
+    (dict(K8=FAKE + 4), B.PKV_ERR_INVALID_ARG),           # misaligned
+    (dict(B=0), B.PKV_ERR_INVALID_ARG),
+    (dict(causal=2), B.PKV_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), B.PKV_ERR_INVALID_ARG),
+    (dict(q_descale=0.0), B.PKV_ERR_INVALID_ARG),
+    (dict(k_descale=math.inf), B.PKV_ERR_INVALID_ARG),
+    (dict(k_descale=-1.0), B.PKV_ERR_INVALID_ARG),
+    (dict(d=64), B.PKV_ERR_UNSUPPORTED),
+    (dict(B=70000), B.PKV_ERR_UNSUPPORTED),
+])
+def test_fp8_prefill_rejects_bad_arguments(kw, status):
+    a = dict(Q8=FAKE, K8=FAKE, V=FAKE, O=FAKE, B=1, H=1, N=16, d=128, causal=1, scale=0.1,
+             q_descale=0.01, k_descale=0.01)
+    a.update(kw)
+    st = B.raw_status("attn_prefill_fp8qk", a["Q8"], a["K8"], a["V"], a["O"], a["B"], a["H"],
+                      a["N"], a["d"], a["causal"], ctypes.c_float(a["scale"]),
+                      ctypes.c_float(a["q_descale"]), ctypes.c_float(a["k_descale"]), None)
+    assert st == status
+
+
+def _append(**kw):
+    a = dict(k_new=FAKE, v_new=FAKE, cu=FAKE, start=FAKE, table=FAKE, maxp=4, S=2, num_new=3,
+             k=FAKE, v=FAKE, P=8, ps=16, H_kv=4, d=128, dtype=B.PKV_BF16)
+    a.update(kw)
+    return B.raw_status("paged_kv_append", a["k_new"], a["v_new"], a["cu"], a["start"], a["table"],
+                        a["maxp"], a["S"], a["num_new"], a["k"], a["v"], a["P"], a["ps"],
+                        a["H_kv"], a["d"], a["dtype"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(num_new=-1), B.PKV_ERR_INVALID_ARG),
+    (dict(S=0), B.PKV_ERR_INVALID_ARG),
+    (dict(ps=8), B.PKV_ERR_INVALID_ARG),
+    (dict(ps=48), B.PKV_ERR_INVALID_ARG),
+    (dict(ps=512), B.PKV_ERR_INVALID_ARG),
+    (dict(dtype=3), B.PKV_ERR_INVALID_ARG),
+    (dict(d=96), B.PKV_ERR_UNSUPPORTED),
+    (dict(k_new=FAKE + 8), B.PKV_ERR_INVALID_ARG),
+    (dict(cu=FAKE + 2), B.PKV_ERR_INVALID_ARG),
+    (dict(table=None), B.PKV_ERR_INVALID_ARG),
+    (dict(P=1 << 24, ps=256), B.PKV_ERR_UNSUPPORTED),       # pool rows beyond 2^31
+    # nothing to write: success before any pointer is looked at or anything launched
+    (dict(num_new=0, k_new=None, v_new=None, cu=None, start=None, table=None), B.PKV_OK),
+])
+def test_append_rejects_bad_arguments(kw, status):
+    assert _append(**kw) == status
+
+
+def _copy(**kw):
+    a = dict(k=FAKE, v=FAKE, src=FAKE, dst=FAKE, n=2, P=8, ps=16, H_kv=4, d=128, dtype=B.PKV_BF16)
+    a.update(kw)
+    return B.raw_status("paged_kv_copy_pages", a["k"], a["v"], a["src"], a["dst"], a["n"], a["P"],
+                        a["ps"], a["H_kv"], a["d"], a["dtype"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(n=-1), B.PKV_ERR_INVALID_ARG),
+    (dict(P=0), B.PKV_ERR_INVALID_ARG),
+    (dict(ps=24), B.PKV_ERR_INVALID_ARG),
+    (dict(dtype=9), B.PKV_ERR_INVALID_ARG),
+    (dict(d=32), B.PKV_ERR_UNSUPPORTED),
+    (dict(v=FAKE + 4), B.PKV_ERR_INVALID_ARG),
+    (dict(src=FAKE + 1), B.PKV_ERR_INVALID_ARG),
+    (dict(n=0, k=None, v=None, src=None, dst=None), B.PKV_OK),
+])
+def test_copy_pages_rejects_bad_arguments(kw, status):
+    assert _copy(**kw) == status
