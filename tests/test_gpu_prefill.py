@@ -64,9 +64,10 @@ def test_dense_large_scores_no_overflow():
 @pytest.mark.parametrize("growth", [7.5, 12.0, 40.0])
 @pytest.mark.parametrize("causal", [True, False])
 def test_running_max_staircase(growth, causal):
-    """Key scores that climb by `growth` (log2 units) per 128-key tile: at 12
-    and 40 every tile moves the row max past the 2^8 rescale threshold, at 7.5
-    none does, and the exponentials reach ~2^7.5 without a rescale."""
+    """Key scores that climb by `growth` (log2 units) per 128-key tile.  At 12
+    and 40 every tile moves the row max more than 8 past the reference max, so
+    O is rescaled at every tile; at 7.5 that happens every second tile, and in
+    between exponentials of up to ~2^7.5 go into P without a rescale."""
     N, d, scale = 1000, 128, 0.088
     g = torch.Generator().manual_seed(77)
     log2e = 1.4426950408889634
