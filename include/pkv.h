@@ -40,6 +40,12 @@
  *   rounded to bf16 before the PV product on the tensor-core path) and
  *   PKV_F32 (float32 in and out, float32 FMA throughout).
  * - Head dimension d: 128 for PKV_BF16; 64 or 128 for PKV_F32.
+ * - Device reset: the library looks up, once per device, the device addresses
+ *   of its own static arrays (the device error word; the scratch of
+ *   paged_decode_noalloc) and keeps them for the life of the process.  A
+ *   cudaDeviceReset, or anything else that destroys and re-creates a device's
+ *   primary context, leaves those addresses stale: do not call the library on
+ *   a device after resetting it in the same process.
  */
 #ifndef PKV_H_
 #define PKV_H_
@@ -191,7 +197,8 @@ PKV_API int paged_attn(const void* q, const void* k_pages, const void* v_pages,
  *   page_size) exceeds PKV_NOALLOC_SCRATCH_BYTES the call returns
  *   PKV_ERR_WORKSPACE and launches nothing.
  * - Set-up: the first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *   (cudaGetSymbolAddress, with that device current) and caches it for the
+ *   life of the process (so not across a device reset, see above); make that
  *   first call before any stream capture.
  * - Sharing: all calls on a device use the same array, which keeps the last
  *   call's contents.  No part of it needs to start at zero (a call writes every

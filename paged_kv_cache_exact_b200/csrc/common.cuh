@@ -128,4 +128,8 @@ cudaError_t launch_copy_pages(const CopyPagesParams& p, cudaStream_t stream);
 // Device address of the library's error word on the current device.
 int device_error_word(unsigned int** out);
 
+// pkv_status of a launcher's result: cudaErrorNotSupported (a configuration
+// with no kernel) -> PKV_ERR_UNSUPPORTED, any other failure -> PKV_ERR_CUDA.
+int cuda_status(cudaError_t e);
+
 }  // namespace pkv

@@ -19,6 +19,8 @@
 //   merged in shared memory, and the splits of a sequence are merged by
 //   `combine_kernel` with the same log-sum-exp algebra (scores are kept in
 //   base-2 units: q is pre-multiplied by scale * log2(e)).
+#include <mutex>
+
 #include "common.cuh"
 
 namespace pkv {
@@ -550,14 +552,20 @@ cudaError_t launch_decode_bf16(const DecodeParams& p, cudaStream_t stream) {
     // grouped heads: one CTA per (split, kv head, 16 query heads, sequence)
     const int n_hg = (p.H / p.H_kv + 15) / 16;
     const size_t smem = kGqaWarps * kWarpSmem + kMaxSplitPages * sizeof(int);
+    // The attribute is per device; callers on several host threads may get
+    // here at once, so the once-per-device record is kept under a lock.
     static bool attr_set[64] = {};
+    static std::mutex attr_mu;
     int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-      e = cudaFuncSetAttribute(decode_gqa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)smem);
-      if (e != cudaSuccess) return e;
-      attr_set[dev] = true;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    {
+      std::lock_guard<std::mutex> lock(attr_mu);
+      if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        e = cudaFuncSetAttribute(decode_gqa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+      }
     }
     // Longer splits than the per-head plan (each CTA now serves up to 16 heads):
     // double while there are still ~8 CTAs per SM.  Fewer splits use less of

@@ -97,6 +97,5 @@ extern "C" PKV_API int paged_decode_noalloc(const void* q, const void* k_pages,
   p.num_pages = num_pages, p.max_pages = max_pages_per_seq, p.max_seq_len = max_seq_len;
   p.split_tokens = split, p.max_splits = nsplit;
   p.scale_log2 = scale * pkv::kLog2e;
-  const cudaError_t e = pkv::launch_decode_bf16(p, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+  return pkv::cuda_status(pkv::launch_decode_bf16(p, static_cast<cudaStream_t>(stream)));
 }

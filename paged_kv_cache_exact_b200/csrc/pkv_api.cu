@@ -39,17 +39,18 @@ int log2i(int x) {
 }
 bool good_scale(float s) { return std::isfinite(s) && s > 0.f; }
 
+}  // namespace
+
+namespace pkv {
+int device_error_word(unsigned int** out) { return error_word(out); }
 int cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return PKV_OK;
   if (e == cudaErrorNotSupported) return PKV_ERR_UNSUPPORTED;
   return PKV_ERR_CUDA;
 }
-
-}  // namespace
-
-namespace pkv {
-int device_error_word(unsigned int** out) { return error_word(out); }
 }  // namespace pkv
+
+using pkv::cuda_status;
 
 extern "C" {
 

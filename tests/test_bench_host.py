@@ -22,6 +22,18 @@ def test_roofline_value_arithmetic():
     assert bench.roofline_value(1e12, 1e9, 0.022, peaks, n_ranks=4) == pytest.approx(200.0)
 
 
+def test_tensor_peak_burst_below_one_second_sustained_above():
+    peaks = {"hbm_gbs": 1000.0, "bf16_tflops": 100.0, "bf16_tflops_sustained": 90.0}
+    # the driver's 20-step region (~23 ms) runs at burst clocks
+    peak, why = bench.tensor_peak(peaks, 0.023)
+    assert peak == 100.0 and "burst" in why and "0.023" in why
+    # a region of seconds of back-to-back work runs under the power cap
+    peak, why = bench.tensor_peak(peaks, 1.2)
+    assert peak == 90.0 and "sustained" in why
+    # the boundary itself counts as sustained
+    assert bench.tensor_peak(peaks, bench.SUSTAINED_AFTER_S)[0] == 90.0
+
+
 def test_peaks_fallback(tmp_path):
     p, src = bench.load_peaks(str(tmp_path / "missing.json"))
     assert src == "fallback" and p["hbm_gbs"] == 6650.0 and p["bf16_tflops"] == 1590.0
