@@ -103,6 +103,28 @@ PKV_API int attn_prefill(const void* Q, const void* K, const void* V, void* O,
                  int dtype, void* stream);
 
 /*
+ * pkv_test_prefill_stalled - test hook for the failure path; not for use in
+ * production.
+ *
+ * The pages have no counterpart: it exists so that tests can make the bf16
+ * prefill's bounded pipeline waits run out without faulting or hanging a GPU.
+ * It runs what attn_prefill runs for dtype PKV_BF16 (same arguments, same
+ * checks), except that every pipeline wait gives up after wait_limit_us
+ * microseconds and the loader of each CTA's first work item never issues the
+ * K load of K/V tile `stall_tile` (0-based).  Every CTA whose first item has
+ * more than stall_tile K/V tiles then records PKV_DEVERR_TIMEOUT, stops,
+ * drains the loads and MMAs it issued, frees its tensor memory and exits;
+ * the output is undefined.  pkv_last_device_error() then returns
+ * PKV_ERR_TIMEOUT, and later calls run normally.
+ *
+ * stall_tile    : >= 0.
+ * wait_limit_us : in [1, 10^7].
+ */
+PKV_API int pkv_test_prefill_stalled(const void* Q, const void* K, const void* V, void* O,
+                                     int B, int H, int N, int d, int causal, float scale,
+                                     int stall_tile, int wait_limit_us, void* stream);
+
+/*
  * attn_prefill_fp8qk - attention with e4m3 (FP8) Q and K, bf16 V and output.
  *
  * Defines: "Flash Attention: Fast, Memory-Efficient Attention for LLMs",

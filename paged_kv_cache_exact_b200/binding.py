@@ -36,6 +36,9 @@ _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_
 
 _lib.attn_prefill.restype = _i
 _lib.attn_prefill.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _vp]
+_lib.pkv_test_prefill_stalled.restype = _i
+_lib.pkv_test_prefill_stalled.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _i,
+                                          _vp]
 _lib.attn_prefill_fp8qk.restype = _i
 _lib.attn_prefill_fp8qk.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _f, _f, _vp]
 _lib.paged_attn_workspace_size.restype = _sz
@@ -115,6 +118,13 @@ def pkv_status_string(status: int) -> str:
 def attn_prefill(Q, K, V, O, B, H, N, d, causal, scale, dtype, stream=None):
     _check("attn_prefill", _lib.attn_prefill(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), B, H, N, d,
                                              int(causal), float(scale), dtype, _stream(stream)))
+
+
+def pkv_test_prefill_stalled(Q, K, V, O, B, H, N, d, causal, scale, stall_tile, wait_limit_us,
+                             stream=None):
+    _check("pkv_test_prefill_stalled", _lib.pkv_test_prefill_stalled(
+        _ptr(Q), _ptr(K), _ptr(V), _ptr(O), B, H, N, d, int(causal), float(scale),
+        int(stall_tile), int(wait_limit_us), _stream(stream)))
 
 
 def attn_prefill_fp8qk(Q8, K8, V, O, B, H, N, d, causal, scale, q_descale, k_descale,

@@ -90,6 +90,13 @@ struct PrefillParams {
   float scale_log2;
   int head_group;   // (batch, head) pairs scheduled together (set by the launcher)
   int fp8_qk;       // Q and K are e4m3 (contiguous only); V and O stay bf16
+  // Failure-path controls; zero (the value-initialised default) means off.
+  // wait_limit_ns bounds every pipeline wait (0 = the default of 2 s).
+  // stall_tile_plus1 = j + 1 is a test hook only: the loader of each CTA's
+  // first work item skips the K load of K/V tile j, so the MMA issuer's wait
+  // for it runs out; the public entry points leave it 0.
+  unsigned long long wait_limit_ns;
+  int stall_tile_plus1;
 };
 
 struct AppendParams {

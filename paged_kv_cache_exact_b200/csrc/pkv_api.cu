@@ -115,6 +115,27 @@ int attn_prefill(const void* Q, const void* K, const void* V, void* O, int B, in
   return PKV_ERR_INVALID_ARG;
 }
 
+int pkv_test_prefill_stalled(const void* Q, const void* K, const void* V, void* O, int B, int H,
+                             int N, int d, int causal, float scale, int stall_tile,
+                             int wait_limit_us, void* stream) {
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return PKV_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1 || (causal != 0 && causal != 1) || !good_scale(scale) ||
+      stall_tile < 0 || wait_limit_us < 1 || wait_limit_us > 10000000)
+    return PKV_ERR_INVALID_ARG;
+  if (d != 128 || B > 65535 || H > 65535) return PKV_ERR_UNSUPPORTED;
+  unsigned int* err = nullptr;
+  if (int r = error_word(&err)) return r;
+  pkv::PrefillParams p{};
+  p.Q = Q, p.K = K, p.V = V, p.O = O;
+  p.err = err;
+  p.B = B, p.H = H, p.H_kv = H, p.q_len = N, p.kv_len = N, p.d = d;
+  p.paged = 0, p.causal = causal;
+  p.scale_log2 = scale * pkv::kLog2e;
+  p.wait_limit_ns = 1000ull * (unsigned long long)wait_limit_us;
+  p.stall_tile_plus1 = stall_tile + 1;
+  return cuda_status(pkv::launch_prefill_bf16(p, static_cast<cudaStream_t>(stream)));
+}
+
 int attn_prefill_fp8qk(const void* Q8, const void* K8, const void* V, void* O, int B, int H,
                        int N, int d, int causal, float scale, float q_descale, float k_descale,
                        void* stream) {

@@ -5,16 +5,26 @@
 // tile, S = Q K^T, a running row max m and row sum l, P = exp(S - m), and the
 // output accumulator rescaled when m moves; S and P never leave the SM.  Its
 // "Flash Attention 2" section's causal skip is kept (tiles past the diagonal
-// are never loaded).  K/V come either from contiguous [B, H_kv, N, d] tensors
-// or, for paged prefill, straight from the pages through the block table
-// ("What is Paged FlashAttention?", "How does it work?"), one TMA box per page.
+// are never loaded, per Q tile).  K/V come either from contiguous
+// [B, H_kv, N, d] tensors or, for paged prefill, straight from the pages
+// through the block table ("What is Paged FlashAttention?", "How does it
+// work?"), one TMA box per page.
 //
 // The B200 design (the pages' H100/SRAM tiling is prior art only):
 //
-// * CTA = two 128-row Q tiles of one (batch, head) sharing every K/V tile.
-//   Warp roles: warps 0-3 and 4-7 are the softmax warpgroups of Q tile 0 and 1
-//   (one thread per row = one TMEM lane), warp 8 issues TMA loads, warp 9
-//   issues tcgen05.mma from one elected lane, warps 10-11 only lend registers.
+// * Work item = two 128-row Q tiles of one (batch, head) sharing every K/V
+//   tile.  The kernel is persistent: it is launched with one CTA per work
+//   item, and a running CTA that nears the end of its item claims the next
+//   unstarted CTA's item through cluster launch control (the hardware cancels
+//   that CTA's launch and hands over its index).  Items keep their launch
+//   order (heaviest causal blocks first, heads grouped for L2), the balance
+//   stays that of the hardware's own greedy placement, and one item's tail
+//   (last PV, epilogue) overlaps the next item's first loads and MMAs
+//   instead of a CTA teardown and launch.
+// * Warp roles: warps 0-3 and 4-7 are the softmax warpgroups of Q tile 0 and
+//   1 (one thread per row = one TMEM lane; each also writes its tile's
+//   output), warp 8 loads (TMA) and claims items, warp 9 issues tcgen05.mma
+//   from one elected lane, warps 10-11 only lend registers.
 // * TMEM (512 columns x 128 lanes x 32 bit): S0 | S1 | O0 | O1, 128 f32 columns
 //   each.  P (bf16) overwrites the first 64 columns of its S once the softmax
 //   has read S into registers, and feeds the PV product straight from TMEM
@@ -24,19 +34,22 @@
 // * Issue order on the MMA warp is S0(j+1) right after PV0(j) and S1(j+1)
 //   right after PV1(j): while the softmax of one Q tile runs, the tensor core
 //   works on the other tile (ping-pong).  tcgen05.mma executes in issue order,
-//   so S_i(j+1) may overwrite P_i(j) once PV_i(j) has been issued.
+//   so S_i(j+1) may overwrite P_i(j) once PV_i(j) has been issued, and the
+//   next item's S_i(0) may follow this item's last PV_i at once.
 // * Online softmax in base 2 with the scale folded into one FFMA; the output
 //   is rescaled only when the running max grows by more than 2^8 (exact: O and
 //   l always share the same reference max, and p stays <= 2^8).
-// * Every mbarrier wait is bounded (about 2 s); on expiry the CTA records
-//   PKV_DEVERR_TIMEOUT, stops issuing work, drains what it already issued and
-//   frees its TMEM.
+// * Every mbarrier wait is bounded; on expiry the CTA records
+//   PKV_DEVERR_TIMEOUT, every role stops, drains what it already issued (TMA
+//   loads, MMAs, an item claim) and the CTA frees its TMEM and exits.
+// * A page id outside the pool is never read: its keys are left out of the
+//   softmax (as the decode kernel does) and its V rows are zeroed, and
+//   PKV_DEVERR_BAD_PAGE is recorded.
 #include <cuda.h>
 
 #include <mutex>
 
 #include "common.cuh"
-#include "exp2_poly.cuh"
 #include "sm100_ptx.cuh"
 
 namespace pkv {
@@ -47,15 +60,15 @@ using namespace sm100;
 constexpr int D = 128;             // head dim
 constexpr int BM = 128;            // rows per Q tile
 constexpr int BN = 128;            // keys per K/V tile
-constexpr int kQTiles = 2;         // Q tiles per CTA
+constexpr int kQTiles = 2;         // Q tiles per work item
 constexpr int kStages = 2;         // K ring and V ring depth
-constexpr int kThreads = 384;      // 3 warpgroups: softmax 0, softmax 1, producer/MMA
+constexpr int kThreads = 384;      // 3 warpgroups: softmax 0, softmax 1, loader/MMA
 // Register split: launched at kLaunchRegs per thread (3 warps per SM
-// sub-partition -> at most 168), then the producer/MMA warpgroup drops to
+// sub-partition -> at most 168), then the loader/MMA warpgroup drops to
 // kRegsSide and both softmax warpgroups rise to kRegsSoftmax.  The split must
 // add up to no more than the launch allocation or setmaxnreg.inc would wait
-// forever, so the host refuses to launch unless the kernel was built with
-// exactly kLaunchRegs registers.
+// forever, so the build fails unless the kernel compiles to exactly
+// kLaunchRegs registers.
 constexpr int kLaunchRegs = 168;
 constexpr int kRegsSoftmax = 208;
 constexpr int kRegsSide = 88;
@@ -63,26 +76,11 @@ static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsSide <= kThreads * kLaunchRegs
               "register split exceeds the launch allocation");
 constexpr int kTileBytes = BM * D * 2;             // 32 KB
 constexpr int kHalfBytes = kTileBytes / 2;         // one 64-column block: 16 KB
-constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
+constexpr uint64_t kDefaultWaitNs = 2000000000ull; // 2 s
 constexpr float kRescaleThreshold = 8.0f;          // log2 units
-// Softmax tuning: one exp2 pair in kPolyEvery goes to the FMA-pipe polynomial
-// (0 = all on MUFU; measured slower at 1/8, 1/4 and 1/2, so off); kSplitP
-// hands P to the PV product in two halves.
-#ifndef PKV_POLY_EVERY
-#define PKV_POLY_EVERY 0
-#endif
-#ifndef PKV_SPLIT_P
-#define PKV_SPLIT_P 1
-#endif
-constexpr int kPolyEvery = PKV_POLY_EVERY;
-// Start the first half's exponentials against the current reference max while
-// the row max is reduced (redo rows whose max grew past the threshold).
-// Measured: +2.5% on the 4x32x4096 prefill, -5..15% on the 32K paged prefill.
-#ifndef PKV_SPEC_EXP
-#define PKV_SPEC_EXP 0
-#endif
-constexpr bool kSpeculativeExp = PKV_SPEC_EXP != 0;
-constexpr bool kSplitP = PKV_SPLIT_P != 0;
+constexpr int kMaskSlots = 4;      // bad-page masks of the K/V tiles in flight
+constexpr int kClaimLead = 3;      // claim the next item this many K/V tiles before the last
+constexpr int kItemReaders = 9;    // warps that read a claimed item id: 8 softmax + MMA
 
 // Shared memory map (offsets from a 1024-aligned base).
 constexpr int kOffQ = 0;
@@ -90,20 +88,27 @@ constexpr int kOffK = kOffQ + kQTiles * kTileBytes;
 constexpr int kOffV = kOffK + kStages * kTileBytes;
 constexpr int kOffBar = kOffV + kStages * kTileBytes;
 enum Bar {
-  kBarQ = 0,
-  kBarKFull = 1,                      // + stage
+  kBarQFull = 0,                      // + q tile
+  kBarQEmpty = kBarQFull + kQTiles,   // + q tile: the item's last S_t has run
+  kBarKFull = kBarQEmpty + kQTiles,   // + stage
   kBarKEmpty = kBarKFull + kStages,   // + stage
   kBarVFull = kBarKEmpty + kStages,
   kBarVEmpty = kBarVFull + kStages,
   kBarSFull = kBarVEmpty + kStages,   // + q tile
-  kBarPHalf = kBarSFull + kQTiles,   // first 64 keys of P in TMEM (+ q tile)
+  kBarPHalf = kBarSFull + kQTiles,    // first 64 keys of P in TMEM (+ q tile)
   kBarPFull = kBarPHalf + kQTiles,    // all of P in TMEM
   kBarODone = kBarPFull + kQTiles,
   kBarVFixed = kBarODone + kQTiles,   // last paged V tile after tail rows are zeroed
-  kBarDrain = kBarVFixed + 1,         // abort path: wait for issued MMAs
+  kBarItem = kBarVFixed + 1,          // + slot: a claimed item id is published
+  kBarItemFree = kBarItem + 2,        // + slot: every reader has taken it
+  kBarClaim = kBarItemFree + 2,       // a launch-control response landed
+  kBarDrain = kBarClaim + 1,          // abort path: wait for issued MMAs
   kNumBars = kBarDrain + 1
 };
-constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
+constexpr int kOffClaim = (kOffBar + kNumBars * 8 + 15) & ~15;   // 16-byte response
+constexpr int kOffItem = kOffClaim + 16;                         // int[2]
+constexpr int kOffMask = kOffItem + 8;                           // uint32[kMaskSlots]
+constexpr int kOffTmemSlot = kOffMask + 4 * kMaskSlots;
 constexpr int kOffAbort = kOffTmemSlot + 4;
 constexpr int kSmemUsed = kOffAbort + 4;
 constexpr int kSmemBytes = kSmemUsed + 1024;       // slack for 1024-byte alignment
@@ -119,22 +124,31 @@ constexpr uint32_t kIdescS8 = make_idesc_e4m3(BM, BN);         // e4m3 Q x e4m3 
 constexpr int kTileBytes8 = BM * D;
 constexpr uint32_t kIdescO = make_idesc_bf16(BM, D, true);    // P (TMEM) x V (MN-major)
 
+// A bad-page mask slot holds the K/V tile's running index (low 24 bits) in
+// bits 8..31 and one bit per page box of the tile (at most 8) in bits 0..7.
+PKV_DEVINLINE uint32_t mask_word(int kv_index, uint32_t bits) {
+  return (static_cast<uint32_t>(kv_index & 0xFFFFFF) << 8) | bits;
+}
+
 struct Geometry {
-  int b, h, kvh, q0, q_len, kv_len, off, n_tiles;
+  int b, h, kvh, q0, kv_len, off;
+  int n[kQTiles];   // K/V tiles Q tile t needs (0: the tile has no rows)
+  int nmax;         // K/V tiles the item loads
+  bool bad_len;
 };
 
-__device__ __forceinline__ Geometry cta_geometry(const PrefillParams& p) {
+// Work item `item` of the launch order: groups of p.head_group (batch, head)
+// pairs; within a group the heaviest causal Q block of every head comes
+// first, then the next heaviest, ...  The host sizes a group so that its K/V
+// (about 32 MB) stays in L2 while its Q blocks run.
+__device__ __forceinline__ Geometry item_geometry(const PrefillParams& p, int item) {
   Geometry g;
-  // 1-D grid, scheduled in groups of p.head_group (batch, head) pairs: within
-  // a group the heaviest causal Q block of every head comes first, then the
-  // next heaviest, ...  The host sizes a group so that its K/V (about 32 MB)
-  // stays in L2 while its Q blocks run; the lightest blocks fill the tail.
   const int m_blocks = (p.q_len + BM * kQTiles - 1) / (BM * kQTiles);
   const int BH = p.B * p.H;
   const int hg = p.head_group;
   const int per_group = hg * m_blocks;
-  const int group = blockIdx.x / per_group;
-  const int r = blockIdx.x - group * per_group;
+  const int group = item / per_group;
+  const int r = item - group * per_group;
   const int heads_here = min(hg, BH - group * hg);
   const int rank = r / heads_here;                  // 0 = heaviest Q block
   const int bh = group * hg + (r - rank * heads_here);
@@ -142,25 +156,34 @@ __device__ __forceinline__ Geometry cta_geometry(const PrefillParams& p) {
   g.h = bh % p.H;
   g.kvh = g.h / (p.H / p.H_kv);
   g.q0 = (m_blocks - 1 - rank) * (BM * kQTiles);
-  g.q_len = p.q_len;
   int kv_len = p.kv_len;
+  g.bad_len = false;
   if (p.paged) {
     kv_len = p.seq_lens[g.b];
     const int cap = min(p.max_seq_len, p.max_pages * p.page_size);
     if (kv_len < p.q_len || kv_len > cap) {
-      if (g.q0 == 0 && g.h == 0 && threadIdx.x == 0) flag_error(p.err, PKV_DEVERR_BAD_LEN);
+      g.bad_len = true;
       kv_len = max(0, min(kv_len, cap));
     }
   }
   g.kv_len = kv_len;
   g.off = kv_len - p.q_len;
-  int n = (kv_len + BN - 1) / BN;
-  if (p.causal) {
-    const int last_row = min(g.q0 + BM * kQTiles - 1, p.q_len - 1);
-    const int last_key = last_row + g.off;      // may be < 0: nothing visible
-    n = last_key < 0 ? 0 : min(n, last_key / BN + 1);
+  const int n_kv = (kv_len + BN - 1) / BN;
+  g.nmax = 0;
+#pragma unroll
+  for (int t = 0; t < kQTiles; ++t) {
+    const int first = g.q0 + t * BM;
+    int n = 0;
+    if (first < p.q_len) {
+      n = n_kv;
+      if (p.causal) {
+        const int last_key = min(first + BM - 1, p.q_len - 1) + g.off;   // < 0: nothing visible
+        n = last_key < 0 ? 0 : min(n_kv, last_key / BN + 1);
+      }
+    }
+    g.n[t] = n;
+    g.nmax = max(g.nmax, n);
   }
-  g.n_tiles = max(n, 0);
   return g;
 }
 
@@ -175,19 +198,21 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const uint32_t sbase = smem_u32(smem);
   auto bar = [&](int i) { return sbase + kOffBar + 8 * i; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
+  volatile int* item_slot = reinterpret_cast<volatile int*>(smem + kOffItem);
+  volatile uint32_t* mask_slot = reinterpret_cast<volatile uint32_t*>(smem + kOffMask);
+  const uint64_t limit_ns = p.wait_limit_ns ? p.wait_limit_ns : kDefaultWaitNs;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const Geometry g = cta_geometry(p);
-  const int n = g.n_tiles;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumBars; ++i) {
-      // P halves: one arrival per softmax thread; everything else: one arrival.
-      const bool per_thread = (i >= kBarPHalf && i < kBarPFull + kQTiles);
-      const uint32_t cnt = per_thread ? 128u : 1u;
+      uint32_t cnt = 1;
+      if (i >= kBarPHalf && i < kBarPFull + kQTiles) cnt = 128;   // one arrival per softmax thread
+      if (i >= kBarItemFree && i < kBarItemFree + 2) cnt = kItemReaders;
       mbar_init(bar(i), cnt);
     }
+    for (int s = 0; s < kMaskSlots; ++s) mask_slot[s] = mask_word(s - kMaskSlots, 0);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -201,76 +226,129 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kOffTmemSlot);
 
   auto fail = [&]() {
-    *abort_flag = 1;
-    flag_error(p.err, PKV_DEVERR_TIMEOUT);
+    if (!*abort_flag) {
+      *abort_flag = 1;
+      flag_error(p.err, PKV_DEVERR_TIMEOUT);
+    }
   };
   // A phase that has already completed costs one try_wait; the abort flag (a
   // shared-memory read) is consulted only once the caller has to wait.
   auto wait = [&](int b, uint32_t parity) -> bool {
     if (mbar_try_wait(bar(b), parity)) return true;
     if (*abort_flag) return false;
-    if (!mbar_wait_bounded(bar(b), parity, kWaitLimitNs)) {
+    if (!mbar_wait_abortable(bar(b), parity, limit_ns, abort_flag)) {
       fail();
       return false;
     }
     return true;
   };
+  auto wwait = [&](int b, uint32_t parity) -> bool {   // warp-uniform result
+    return __all_sync(0xffffffffu, wait(b, parity));
+  };
+  // Item id number `kk` claimed after the CTA's own (a whole warp calls this):
+  // wait until the loader publishes it, read it, and release the slot.  -1 =
+  // no item left; -2 = the CTA is aborting.
+  auto read_item = [&](int kk) -> int {
+    if (!wwait(kBarItem + (kk & 1), (kk >> 1) & 1)) return -2;
+    const int v = item_slot[kk & 1];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar(kBarItemFree + (kk & 1)));
+    return v;
+  };
 
   if (warp >= 8) regs_decrease<kRegsSide>();
 
   if (warp == 8) {
-    // ------------------------------------------------------------ producer --
-    // The warp runs the loop converged.  Contiguous tiles and pages of >= 128
-    // tokens take one TMA box per 64-column block, issued by lane 0; shorter
-    // pages take one box per page per block, and lane i resolves page i of the
-    // tile and issues its boxes, so the boxes of a tile are issued in parallel
-    // (one thread issuing 16 of them per K or V tile could not keep ahead of
-    // the tensor core).  Each table entry is read once and serves K and V.
-    if (n > 0) {
-      if (lane == 0) {
-        prefetch_tmap(&tmQ);
-        prefetch_tmap(&tmK);
-        prefetch_tmap(&tmV);
-        const int qc2 = g.b * p.H + g.h;
-        mbar_arrive_expect_tx(bar(kBarQ), kQTiles * (kFp8QK ? kTileBytes8 : kTileBytes));
-        for (int t = 0; t < kQTiles; ++t)
+    // ------------------------------------------------------------- loader --
+    // The warp runs converged.  Contiguous tiles and pages of >= 128 tokens
+    // take one TMA box per 64-column block, issued by lane 0; shorter pages
+    // take one box per page per block, and lane i resolves page i of the tile
+    // and issues its boxes, so the boxes of a tile are issued in parallel.
+    // Each table entry is read once and serves K and V.
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+    }
+    const uint32_t qk_bytes = kFp8QK ? kTileBytes8 : kTileBytes;
+    const int rows_per_box = kPaged ? min(p.page_size, BN) : BN;
+    const bool box_per_page = kPaged && rows_per_box < BN;
+    int kv_it = 0, tail_it = 0, claims = 0;
+    int q_it[kQTiles] = {0, 0};
+    // Loads issued whose completion nobody has seen yet (for the abort
+    // drain), two bits per barrier: bit 0 = pending, bit 1 = its phase parity.
+    // Fields: K stage s at 2s, V stage s at 4 + 2s, Q tile t at 8 + 2t.
+    uint32_t pend = 0;
+    auto set_pend = [&](int field, uint32_t parity) {
+      pend = (pend & ~(3u << (2 * field))) | ((1u | (parity << 1)) << (2 * field));
+    };
+    auto clear_pend = [&](int field) { pend &= ~(3u << (2 * field)); };
+    bool pend_claim = false;
+    bool claim_live = true;     // after a failed claim no further claim may be made
+    bool ok = true;
+    int item = blockIdx.x;
+    for (int k = 0; ok && item >= 0; ++k) {
+      const Geometry g = item_geometry(p, item);
+      if (g.bad_len && g.q0 == 0 && g.h == 0 && lane == 0) flag_error(p.err, PKV_DEVERR_BAD_LEN);
+      const int nmax = g.nmax;
+      bool claimed = false;
+      auto claim = [&]() {
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar(kBarClaim), 16);
+          clc_try_cancel(sbase + kOffClaim, bar(kBarClaim));
+        }
+        __syncwarp();
+        claimed = true;
+        pend_claim = true;
+      };
+      auto load_q = [&](int t) -> bool {
+        if (!wwait(kBarQEmpty + t, (q_it[t] & 1) ^ 1)) return false;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar(kBarQFull + t), qk_bytes);
           for (int c = 0; c < (kFp8QK ? 1 : 2); ++c)
             tma_load_3d(sbase + kOffQ + t * kTileBytes + c * kHalfBytes, &tmQ, c * 64,
-                        g.q0 + t * BM, qc2, bar(kBarQ));
-      }
-      auto wwait = [&](int b, uint32_t parity) -> bool {
-        return __all_sync(0xffffffffu, wait(b, parity));
+                        g.q0 + t * BM, g.b * p.H + g.h, bar(kBarQFull + t));
+        }
+        __syncwarp();
+        set_pend(4 + t, q_it[t] & 1);
+        return true;
       };
-      int last_k = -1, last_v = -1;                  // last tile whose K / V load was issued
-      const int rows_per_box = kPaged ? min(p.page_size, BN) : BN;
-      const bool box_per_page = kPaged && rows_per_box < BN;
+      if (g.n[0] > 0) ok = load_q(0);
       const int n_valid_pages = kPaged ? (g.kv_len + p.page_size - 1) >> p.page_shift : 0;
       const int32_t* trow = p.block_table + (size_t)g.b * p.max_pages;
-      bool ok = true;
-      for (int j = 0; j < n && ok; ++j) {
-        const int st = j % kStages;
-        const uint32_t ph = (j / kStages) & 1;
+      for (int j = 0; j < nmax && ok; ++j) {
+        if (!claimed && claim_live && j >= nmax - kClaimLead) claim();
+        const int it = kv_it + j;
+        const int st = it % kStages;
+        const uint32_t ph = (it / kStages) & 1;
         const int k0 = j * BN;
         // boxes of this tile that hold tokens of the sequence (never past its last page)
         const int nbox = kPaged ? min(BN / rows_per_box, n_valid_pages - (k0 >> p.page_shift)) : 1;
-        const uint32_t bytes = kPaged ? nbox * rows_per_box * 256 : kTileBytes;
-        // this lane's box: first token row of its page slice in the pool
-        const int mine = box_per_page ? lane : 0;
+        const int mine = box_per_page ? lane : 0;     // this lane's box
         int row = 0;
+        bool good = true;
         if (kPaged && mine < nbox) {
-          int phys = trow[(k0 + mine * rows_per_box) >> p.page_shift];
-          if (phys < 0 || phys >= p.num_pages) {     // never read outside the pool
-            flag_error(p.err, PKV_DEVERR_BAD_PAGE);
-            phys = 0;
-          }
+          const int phys = trow[(k0 + mine * rows_per_box) >> p.page_shift];
+          good = phys >= 0 && phys < p.num_pages;     // never read outside the pool
           row = phys * p.page_size + ((k0 + mine * rows_per_box) & (p.page_size - 1));
         }
-        const bool issues = box_per_page ? lane < nbox : lane == 0;
+        const bool in_tile = box_per_page ? lane < nbox : lane == 0;
+        const uint32_t bad = kPaged ? __ballot_sync(0xffffffffu, in_tile && !good) : 0u;
+        // bad boxes: bit b = box b (box_per_page), or bit 0 = the whole tile
+        const uint32_t bad_boxes = box_per_page ? bad : (bad ? 1u : 0u);
+        const int n_good = (kPaged ? nbox : 1) - __popc(bad_boxes);
+        const uint32_t bytes = kPaged ? n_good * rows_per_box * 256 : qk_bytes;
+        const bool issues = in_tile && good;
+        if (kPaged && bad && lane == 0) flag_error(p.err, PKV_DEVERR_BAD_PAGE);
+
         ok = wwait(kBarKEmpty + st, ph ^ 1);
         if (!ok) break;
+        clear_pend(st);
+        if (kPaged && lane == 0) mask_slot[it % kMaskSlots] = mask_word(it, bad_boxes);
+        const bool stall = p.stall_tile_plus1 == j + 1 && k == 0;   // test hook: K(j) never lands
         if (lane == 0) mbar_arrive_expect_tx(bar(kBarKFull + st), kFp8QK ? kTileBytes8 : bytes);
         __syncwarp();
-        if (issues) {
+        if (issues && !stall) {
           for (int c = 0; c < (kFp8QK ? 1 : 2); ++c) {
             const uint32_t dst = sbase + kOffK + st * kTileBytes + c * kHalfBytes;
             if (kPaged)
@@ -279,10 +357,28 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
               tma_load_3d(dst, &tmK, c * 64, k0, g.b * p.H_kv + g.kvh, bar(kBarKFull + st));
           }
         }
-        last_k = j;
+        if (!stall && __any_sync(0xffffffffu, issues)) set_pend(st, ph);
+        if (j == 0 && g.n[1] > 0) {
+          ok = load_q(1);
+          if (!ok) break;
+        }
+
         ok = wwait(kBarVEmpty + st, ph ^ 1);
         if (!ok) break;
-        if (lane == 0) mbar_arrive_expect_tx(bar(kBarVFull + st), bytes);
+        clear_pend(2 + st);
+        if (kPaged && bad_boxes) {
+          // V rows of skipped boxes must be zero: P is 0 there, but 0 * NaN = NaN.
+          uint8_t* vt = smem + kOffV + st * kTileBytes;
+          for (int idx = lane; idx < BN * 16; idx += 32) {   // 16 x 16 B per row (2 blocks)
+            const int r = idx / 16, part = idx % 16;
+            if (!((bad_boxes >> (box_per_page ? r / rows_per_box : 0)) & 1)) continue;
+            *reinterpret_cast<uint4*>(vt + (part / 8) * kHalfBytes + r * 128 + (part % 8) * 16) =
+                make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive_expect_tx(bar(kBarVFull + st), kPaged ? bytes : kTileBytes);
         __syncwarp();
         if (issues) {
           for (int c = 0; c < 2; ++c) {
@@ -293,43 +389,64 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
               tma_load_3d(dst, &tmV, c * 64, k0, g.b * p.H_kv + g.kvh, bar(kBarVFull + st));
           }
         }
-        last_v = j;
+        if (__any_sync(0xffffffffu, issues)) set_pend(2 + st, ph);
       }
-      if (!ok && lane == 0) {
-        // Drain loads already in flight before the CTA's shared memory goes away.
-        for (int jj = max(0, last_k - 1); jj <= last_k; ++jj)
-          mbar_wait_bounded(bar(kBarKFull + jj % kStages), (jj / kStages) & 1, kWaitLimitNs);
-        for (int jj = max(0, last_v - 1); jj <= last_v; ++jj)
-          mbar_wait_bounded(bar(kBarVFull + jj % kStages), (jj / kStages) & 1, kWaitLimitNs);
-      }
-    }
-    // Paged, last tile partial: rows past kv_len (poisoned tails, unread pages)
-    // must be zero in V, since P = 0 there but 0 * NaN is NaN.  The whole warp
-    // zeroes them once the tile has landed, then releases it to the MMA warp.
-    if (kPaged && n > 0) {
-      const int j = n - 1;
-      const int valid = g.kv_len - j * BN;
-      if (valid < BN) {
-        __syncwarp();
-        const int st = j % kStages;
-        bool ok = !*abort_flag;
-        if (lane == 0 && ok) ok = mbar_wait_bounded(bar(kBarVFull + st), (j / kStages) & 1, kWaitLimitNs);
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        if (ok) {
-          uint8_t* vt = smem + kOffV + st * kTileBytes;
-          const int nrows = BN - valid;
-          for (int idx = lane; idx < nrows * 16; idx += 32) {       // 16 x 16 B per row (2 blocks)
-            const int r = valid + idx / 16, part = idx % 16;
-            *reinterpret_cast<uint4*>(vt + (part / 8) * kHalfBytes + r * 128 + (part % 8) * 16) =
-                make_uint4(0, 0, 0, 0);
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(kBarVFixed));
-        } else if (lane == 0) {
-          fail();
+      if (!ok) break;
+      if (!claimed && claim_live) claim();
+      // Paged, last tile partial: rows past kv_len (poisoned tails, unread
+      // pages) must be zero in V, since P = 0 there but 0 * NaN is NaN.  The
+      // whole warp zeroes them once the tile has landed, then releases it to
+      // the MMA warp.
+      if (kPaged && nmax > 0 && g.kv_len - (nmax - 1) * BN < BN) {
+        const int it = kv_it + nmax - 1;
+        const int st = it % kStages;
+        const int valid = g.kv_len - (nmax - 1) * BN;
+        if ((pend >> (2 * (2 + st))) & 1) ok = wwait(kBarVFull + st, (it / kStages) & 1);
+        if (!ok) break;
+        clear_pend(2 + st);
+        uint8_t* vt = smem + kOffV + st * kTileBytes;
+        for (int idx = lane; idx < (BN - valid) * 16; idx += 32) {   // 16 x 16 B per row
+          const int r = valid + idx / 16, part = idx % 16;
+          *reinterpret_cast<uint4*>(vt + (part / 8) * kHalfBytes + r * 128 + (part % 8) * 16) =
+              make_uint4(0, 0, 0, 0);
         }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kBarVFixed));
+        ++tail_it;
       }
+      // The next item: the one the claim returned, or none.
+      int next = -1;
+      if (claim_live) {
+        ok = wwait(kBarClaim, claims & 1);
+        if (!ok) break;
+        pend_claim = false;
+        ++claims;
+        next = __shfl_sync(0xffffffffu, lane == 0 ? clc_cancelled_x(sbase + kOffClaim) : 0, 0);
+        if (next < 0) claim_live = false;
+      }
+      ok = wwait(kBarItemFree + (k & 1), ((k >> 1) & 1) ^ 1);
+      if (!ok) break;
+      if (lane == 0) {
+        item_slot[k & 1] = next;
+        mbar_arrive(bar(kBarItem + (k & 1)));
+      }
+      __syncwarp();
+      kv_it += nmax;
+#pragma unroll
+      for (int t = 0; t < kQTiles; ++t) q_it[t] += g.n[t] > 0;
+      item = next;
+    }
+    if (!ok && lane == 0) {
+      // Drain loads (and a claim) in flight before the CTA's shared memory goes away.
+      // field f: barrier kBarKFull + s (f = s), kBarVFull + s (f = 2 + s) or
+      // kBarQFull + t (f = 4 + t)
+      const int field_bar[6] = {kBarKFull, kBarKFull + 1, kBarVFull, kBarVFull + 1, kBarQFull,
+                                kBarQFull + 1};
+      for (int f = 0; f < 6; ++f)
+        if ((pend >> (2 * f)) & 1)
+          mbar_wait_bounded(bar(field_bar[f]), (pend >> (2 * f + 1)) & 1, limit_ns);
+      if (pend_claim) mbar_wait_bounded(bar(kBarClaim), claims & 1, limit_ns);
     }
   } else if (warp == 9) {
     // ----------------------------------------------------------------- MMA --
@@ -340,41 +457,53 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // stage so that an issue costs one add and the MMA: a 128x128x16 MMA
     // retires in 64 cycles, less than a descriptor rebuild takes.  The warp
     // runs converged and one elected lane issues.
-    auto wwait = [&](int b, uint32_t parity) -> bool {
-      return __all_sync(0xffffffffu, wait(b, parity));
-    };
-    if (n > 0) {
-      const bool last_fix = kPaged && (g.kv_len - (n - 1) * BN) < BN;
-      const uint64_t dq0 = make_sdesc(sbase + kOffQ, 16, 1024);
-      const uint64_t dq1 = make_sdesc(sbase + kOffQ + kTileBytes, 16, 1024);
-      const uint64_t dk0 = make_sdesc(sbase + kOffK, 16, 1024);
-      const uint64_t dk1 = make_sdesc(sbase + kOffK + kTileBytes, 16, 1024);
-      const uint64_t dv0 = make_sdesc(sbase + kOffV, kHalfBytes, 1024);
-      const uint64_t dv1 = make_sdesc(sbase + kOffV + kTileBytes, kHalfBytes, 1024);
-      const bool leader = elect_one();
+    const uint64_t dq[kQTiles] = {make_sdesc(sbase + kOffQ, 16, 1024),
+                                  make_sdesc(sbase + kOffQ + kTileBytes, 16, 1024)};
+    const uint64_t dk0 = make_sdesc(sbase + kOffK, 16, 1024);
+    const uint64_t dk1 = make_sdesc(sbase + kOffK + kTileBytes, 16, 1024);
+    const uint64_t dv0 = make_sdesc(sbase + kOffV, kHalfBytes, 1024);
+    const uint64_t dv1 = make_sdesc(sbase + kOffV + kTileBytes, kHalfBytes, 1024);
+    const bool leader = elect_one();
+    int kv_it = 0, tail_it = 0;
+    int q_it[kQTiles] = {0, 0}, p_it[kQTiles] = {0, 0};
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int item = k == 0 ? blockIdx.x : read_item(k - 1);
+      if (item == -2) ok = false;
+      if (item < 0) break;
+      const Geometry g = item_geometry(p, item);
+      const int nmax = g.nmax;
+      if (nmax == 0) continue;
+      const bool last_fix = kPaged && g.kv_len - (nmax - 1) * BN < BN;
+      int s_left[kQTiles] = {g.n[0], g.n[1]};
+      auto commit = [&](int b) {
+        if (leader) mma_commit(bar(b));
+        __syncwarp();
+      };
+      // S_t = Q_t K(j)^T for K/V tile j of this item (K(j) has landed).
       auto issue_s = [&](int t, int j) {
-        const uint64_t dk = (j % kStages) ? dk1 : dk0;
-        const uint64_t dq = t ? dq1 : dq0;
+        const uint64_t dk = ((kv_it + j) % kStages) ? dk1 : dk0;
         const uint32_t tS = tmem + kColS + 128 * t;
         if (leader) {
           if (kFp8QK) {
 #pragma unroll
             for (int kk = 0; kk < D / 32; ++kk)     // K = 32 e4m3 (32 bytes) per MMA
-              mma_ss_f8(tS, dq + ((kk * 32) >> 4), dk + ((kk * 32) >> 4), kIdescS8, kk > 0);
+              mma_ss_f8(tS, dq[t] + ((kk * 32) >> 4), dk + ((kk * 32) >> 4), kIdescS8, kk > 0);
           } else {
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint64_t koff = ((kk / 4) * kHalfBytes + (kk % 4) * 32) >> 4;
-              mma_ss(tS, dq + koff, dk + koff, kIdescS, kk > 0);
+              mma_ss(tS, dq[t] + koff, dk + koff, kIdescS, kk > 0);
             }
           }
           mma_commit(bar(kBarSFull + t));
+          if (--s_left[t] == 0) mma_commit(bar(kBarQEmpty + t));   // Q_t may be reloaded
         }
         __syncwarp();
       };
       // O_t += P_t V over key steps [kk0, kk0 + 4): P arrives in two halves.
       auto issue_pv_half = [&](int t, int j, int kk0) {
-        const uint64_t dv = (j % kStages) ? dv1 : dv0;
+        const uint64_t dv = ((kv_it + j) % kStages) ? dv1 : dv0;
         const uint32_t tS = tmem + kColS + 128 * t;
         const uint32_t tO = tmem + kColO + 128 * t;
         if (leader) {
@@ -385,160 +514,204 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         __syncwarp();
       };
+      auto wait_k = [&](int j) {
+        const int it = kv_it + j;
+        return wwait(kBarKFull + it % kStages, (it / kStages) & 1);
+      };
       // PV_t(j).  With want_k the next K tile is checked while the second half
       // of P is still being written, so that PV's second half and S_t(j+1)
       // issue back to back once P is complete.
-      auto issue_pv = [&](int t, int j, bool want_k = false) -> bool {
-        if (kSplitP) {
-          if (!wwait(kBarPHalf + t, j & 1)) return false;
-          tc_fence_after();
-          issue_pv_half(t, j, 0);
-        }
-        if (want_k && !wwait(kBarKFull + (j + 1) % kStages, ((j + 1) / kStages) & 1)) return false;
-        if (!wwait(kBarPFull + t, j & 1)) return false;
+      auto issue_pv = [&](int t, int j, bool want_k) -> bool {
+        if (!wwait(kBarPHalf + t, p_it[t] & 1)) return false;
         tc_fence_after();
-        if (!kSplitP) issue_pv_half(t, j, 0);
+        issue_pv_half(t, j, 0);
+        if (want_k && !wait_k(j + 1)) return false;
+        if (!wwait(kBarPFull + t, p_it[t] & 1)) return false;
+        tc_fence_after();
         issue_pv_half(t, j, BN / 32);
         if (leader) mma_commit(bar(kBarODone + t));
         __syncwarp();
+        ++p_it[t];
         return true;
       };
-      auto commit = [&](int b) {
-        if (leader) mma_commit(bar(b));
-        __syncwarp();
-      };
-      bool ok = wwait(kBarQ, 0) && wwait(kBarKFull + 0, 0);
-      if (ok) {
+
+      ok = wait_k(0);
+#pragma unroll
+      for (int t = 0; t < kQTiles; ++t) {
+        if (!ok || g.n[t] == 0) continue;
+        ok = wwait(kBarQFull + t, q_it[t] & 1);
+        if (!ok) continue;
         tc_fence_after();
-        issue_s(0, 0);
-        issue_s(1, 0);
-        commit(kBarKEmpty + 0);
+        issue_s(t, 0);
       }
-      for (int j = 0; j < n && ok; ++j) {
-        const int st = j % kStages;
-        if (last_fix && j == n - 1)
-          ok = wwait(kBarVFixed, 0);
+      if (ok) commit(kBarKEmpty + kv_it % kStages);
+      for (int j = 0; j < nmax && ok; ++j) {
+        const int it = kv_it + j;
+        const int st = it % kStages;
+        if (last_fix && j == nmax - 1)
+          ok = wwait(kBarVFixed, tail_it & 1);
         else
-          ok = wwait(kBarVFull + st, (j / kStages) & 1);
-        ok = ok && issue_pv(0, j, j + 1 < n);
-        if (!ok) break;
-        if (j + 1 < n) {
-          tc_fence_after();
-          issue_s(0, j + 1);
+          ok = wwait(kBarVFull + st, (it / kStages) & 1);
+        bool have_k = false;
+#pragma unroll
+        for (int t = 0; t < kQTiles; ++t) {
+          if (!ok || j >= g.n[t]) continue;
+          const bool more = j + 1 < g.n[t];
+          ok = issue_pv(t, j, more && !have_k);
+          if (!ok) continue;
+          have_k = have_k || more;
+          if (more) {
+            tc_fence_after();
+            issue_s(t, j + 1);
+          }
         }
-        ok = issue_pv(1, j);
         if (!ok) break;
         commit(kBarVEmpty + st);
-        if (j + 1 < n) {
-          issue_s(1, j + 1);
-          commit(kBarKEmpty + (j + 1) % kStages);
-        }
+        if (j + 1 < nmax) commit(kBarKEmpty + (it + 1) % kStages);
       }
-      if (!ok) {
-        // Let every MMA already issued finish before TMEM is released.
-        commit(kBarDrain);
-        mbar_wait_bounded(bar(kBarDrain), 0, kWaitLimitNs);
-      }
+      kv_it += nmax;
+      tail_it += last_fix;
+#pragma unroll
+      for (int t = 0; t < kQTiles; ++t) q_it[t] += g.n[t] > 0;
+    }
+    if (!ok) {
+      // Let every MMA already issued finish before TMEM is released.
+      if (leader) mma_commit(bar(kBarDrain));
+      __syncwarp();
+      mbar_wait_bounded(bar(kBarDrain), 0, limit_ns);
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------- softmax --
     regs_increase<kRegsSoftmax>();
     const int t = warp >> 2;                         // Q tile of this warpgroup
     const int r = threadIdx.x & 127;                 // row in tile = TMEM lane
-    const int row = g.q0 + t * BM + r;               // query row
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_addr + kColS + 128 * t;
     const uint32_t tO = tmem + lane_addr + kColO + 128 * t;
     const float c = p.scale_log2;
-    const int limit = p.causal ? min(row + g.off, g.kv_len - 1) : g.kv_len - 1;
-
-    float m_ref = -INFINITY, l = 0.f;
+    const int box_shift = kPaged ? min(p.page_shift, 7) : 7;   // log2(rows per page box)
+    int kv_it = 0, s_it = 0;
     bool ok = true;
-    // tcgen05.ld/st are warp-collective: every branch around them is warp-uniform.
-    for (int j = 0; j < n; ++j) {
-      ok = wait(kBarSFull + t, j & 1);
-      if (ok && j > 0) ok = wait(kBarODone + t, (j - 1) & 1);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t s[128];
+    for (int k = 0; ok; ++k) {
+      const int item = k == 0 ? blockIdx.x : read_item(k - 1);
+      if (item == -2) ok = false;
+      if (item < 0) break;
+      const Geometry g = item_geometry(p, item);
+      const int n = g.n[t];
+      const int row = g.q0 + t * BM + r;             // query row
+      const int limit = p.causal ? min(row + g.off, g.kv_len - 1) : g.kv_len - 1;
+      float m_ref = -INFINITY, l = 0.f;
+      // tcgen05.ld/st are warp-collective: every branch around them is warp-uniform.
+      for (int j = 0; j < n; ++j) {
+        ok = __all_sync(0xffffffffu, wait(kBarSFull + t, s_it & 1));
+        if (!ok) break;
+        ++s_it;
+        uint32_t bad_keys[4] = {0u, 0u, 0u, 0u};      // keys of pages outside the pool
+        if (kPaged) {
+          // Keys of pages outside the pool are left out (their K rows were
+          // never loaded).  The loader wrote this tile's mask before its K load.
+          const int it = kv_it + j;
+          uint32_t w = mask_slot[it % kMaskSlots];
+          if ((w >> 8) != static_cast<uint32_t>(it & 0xFFFFFF)) {
+            const uint64_t t0 = globaltimer_ns();
+            while ((w >> 8) != static_cast<uint32_t>(it & 0xFFFFFF)) {
+              if (*abort_flag || globaltimer_ns() - t0 > limit_ns) {
+                fail();
+                break;
+              }
+              w = mask_slot[it % kMaskSlots];
+            }
+          }
+          if (!__all_sync(0xffffffffu, !*abort_flag)) {   // the mask wait gave up
+            ok = false;
+            break;
+          }
+          const uint32_t bad_boxes = w & 0xFFu;           // same on every lane
+          if (bad_boxes) {
+            // A box is 16 keys (16-token pages: two boxes per word) or a
+            // multiple of 32 keys (one box covers whole words).
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t (&sub)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[32 * ch]);
-        tmem_ld32(tS + 32 * ch, sub);
-      }
-      tmem_wait_ld();
-      const int k0 = j * BN;
-      const bool masked = k0 + BN - 1 > limit;       // diagonal or tail tile
-      if (masked) {
+            for (int q = 0; q < 4; ++q) {
+              if (box_shift == 4)
+                bad_keys[q] = (((bad_boxes >> (2 * q)) & 1u) ? 0x0000FFFFu : 0u) |
+                              (((bad_boxes >> (2 * q + 1)) & 1u) ? 0xFFFF0000u : 0u);
+              else
+                bad_keys[q] = ((bad_boxes >> ((32 * q) >> box_shift)) & 1u) ? 0xFFFFFFFFu : 0u;
+            }
+          }
+        }
+        tc_fence_after();
+        uint32_t s[128];
 #pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (k0 + i > limit) s[i] = __float_as_uint(-INFINITY);
-      }
-      // row max: eight chains of 3-input max (dependency depth 8)
-      float am[8];
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t (&sub)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[32 * ch]);
+          tmem_ld32(tS + 32 * ch, sub);
+        }
+        tmem_wait_ld();
+        const int k0 = j * BN;
+        // Diagonal or tail tile, or keys of a bad page: one masking pass over
+        // a bit per key (bit b of word q = key k0 + 32 q + b is hidden).
+        const bool masked = k0 + BN - 1 > limit ||
+                            (kPaged && (bad_keys[0] | bad_keys[1] | bad_keys[2] | bad_keys[3]));
+        if (masked) {
 #pragma unroll
-      for (int a = 0; a < 8; ++a) am[a] = __uint_as_float(s[a]);
+          for (int q = 0; q < 4; ++q) {
+            const int first_hidden = limit + 1 - (k0 + 32 * q);     // keys >= this are hidden
+            uint32_t hide = first_hidden <= 0 ? 0xFFFFFFFFu
+                          : first_hidden >= 32 ? 0u : (0xFFFFFFFFu << first_hidden);
+            if (kPaged) hide |= bad_keys[q];
 #pragma unroll
-      for (int i = 8; i + 16 <= 128; i += 16) {        // elements 8 .. 119
+            for (int b = 0; b < 32; ++b)
+              if ((hide >> b) & 1u) s[32 * q + b] = __float_as_uint(-INFINITY);
+          }
+        }
+        // row max: eight chains of 3-input max (dependency depth 8)
+        float am[8];
 #pragma unroll
-        for (int a = 0; a < 8; ++a)
-          am[a] = max3(am[a], __uint_as_float(s[i + 2 * a]), __uint_as_float(s[i + 2 * a + 1]));
-      }
+        for (int a = 0; a < 8; ++a) am[a] = __uint_as_float(s[a]);
 #pragma unroll
-      for (int a = 0; a < 8; ++a) am[a] = fmaxf(am[a], __uint_as_float(s[120 + a]));   // 120 .. 127
-      const float mx = max3(max3(am[0], am[1], am[2]), max3(am[3], am[4], am[5]),
-                            fmaxf(am[6], am[7]));
-      // The first half's exponentials are computed against the current
-      // reference max while the row max above is still being reduced (the two
-      // are independent, so they interleave); they are redone only in rows
-      // whose max grew past the rescale threshold, which after the first tile
-      // is rare.  Masked tiles stay on MUFU (exact zeros); elsewhere
-      // kPolyEvery selects the share of pairs on the FMA-pipe polynomial.
-      const bool poly = !__any_sync(0xffffffffu, masked);
-      const uint64_t c2 = f2(c, c);
-      uint64_t acc[4];
-      auto exp_half = [&](int ch, float neg_m, uint32_t (&pk)[32]) {
-        const uint64_t nm2 = f2(neg_m, neg_m);
+        for (int i = 8; i + 16 <= 128; i += 16) {        // elements 8 .. 119
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int e = 64 * ch + 2 * i;
-          const uint64_t x2 = fma2(f2(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), c2, nm2);
-          float p0, p1;
-          if (kPolyEvery > 0 && poly && (i % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
-            exp2_poly_pair(x2, p0, p1);
-          } else {
+          for (int a = 0; a < 8; ++a)
+            am[a] = max3(am[a], __uint_as_float(s[i + 2 * a]), __uint_as_float(s[i + 2 * a + 1]));
+        }
+#pragma unroll
+        for (int a = 0; a < 8; ++a) am[a] = fmaxf(am[a], __uint_as_float(s[120 + a]));   // 120 .. 127
+        const float mx = max3(max3(am[0], am[1], am[2]), max3(am[3], am[4], am[5]),
+                              fmaxf(am[6], am[7]));
+        const uint64_t c2 = f2(c, c);
+        uint64_t acc[4];
+        auto exp_half = [&](int ch, float neg_m, uint32_t (&pk)[32]) {
+          const uint64_t nm2 = f2(neg_m, neg_m);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int e = 64 * ch + 2 * i;
+            const uint64_t x2 = fma2(f2(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), c2, nm2);
             float x0, x1;
             unf2(x2, x0, x1);
-            p0 = ex2(x0);
-            p1 = ex2(x1);
+            const float p0 = ex2(x0);
+            const float p1 = ex2(x1);
+            acc[i & 3] = add2(acc[i & 3], f2(p0, p1));
+            pk[i] = pack_bf16x2(p0, p1);
           }
-          acc[i & 3] = add2(acc[i & 3], f2(p0, p1));
-          pk[i] = pack_bf16x2(p0, p1);
-        }
-      };
+        };
 #pragma unroll
-      for (int a = 0; a < 4; ++a) acc[a] = f2(0.f, 0.f);
-      uint32_t pk[32];
-      if (kSpeculativeExp) exp_half(0, (m_ref == -INFINITY) ? 0.f : -m_ref, pk);
-      const float m_tile = mx * c;                  // running max in log2 units
-      float alpha = 1.f;
-      bool rescale = false;
-      if (m_tile > m_ref + kRescaleThreshold || (m_ref == -INFINITY && m_tile != -INFINITY)) {
-        alpha = ex2(m_ref - m_tile);               // m_ref = -inf -> 0
-        m_ref = m_tile;
-        rescale = true;
-      }
-      const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
-      if (!kSpeculativeExp) exp_half(0, neg_m, pk);
-      if (__any_sync(0xffffffffu, rescale)) {
-        if (kSpeculativeExp && rescale) {          // redo this row's first half
-#pragma unroll
-          for (int a = 0; a < 4; ++a) acc[a] = f2(0.f, 0.f);
-          exp_half(0, neg_m, pk);
+        for (int a = 0; a < 4; ++a) acc[a] = f2(0.f, 0.f);
+        uint32_t pk[32];
+        const float m_tile = mx * c;                  // running max in log2 units
+        float alpha = 1.f;
+        bool rescale = false;
+        if (m_tile > m_ref + kRescaleThreshold || (m_ref == -INFINITY && m_tile != -INFINITY)) {
+          alpha = ex2(m_ref - m_tile);               // m_ref = -inf -> 0
+          m_ref = m_tile;
+          rescale = true;
         }
-        // O must be rescaled before PV(j) may start, i.e. before any P is handed over.
-        if (j > 0) {                               // alpha = 1 in rows that keep m
+        const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+        exp_half(0, neg_m, pk);
+        if (__any_sync(0xffffffffu, rescale) && j > 0) {
+          // O must be rescaled before PV(j) may start, i.e. before any P is
+          // handed over; PV(j-1) has completed (S(j) was issued after it).
+          // alpha = 1 in rows that keep m.
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
             uint32_t o[32];
@@ -549,52 +722,57 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             tmem_st32(tO + 32 * ch, o);
           }
         }
-      }
-      tmem_st32(tS, pk);
-      if (kSplitP) {                               // first half of P: PV(j) may start
-        tmem_wait_st();
+        tmem_st32(tS, pk);
+        tmem_wait_st();                              // first half of P: PV(j) may start
         tc_fence_before();
         mbar_arrive(bar(kBarPHalf + t));
+        exp_half(1, neg_m, pk);
+        tmem_st32(tS + 32, pk);
+        float s0, s1;
+        unf2(add2(add2(acc[0], acc[1]), add2(acc[2], acc[3])), s0, s1);
+        l = l * alpha + (s0 + s1);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(kBarPFull + t));
       }
-      exp_half(1, neg_m, pk);
-      tmem_st32(tS + 32, pk);
-      float s0, s1;
-      unf2(add2(add2(acc[0], acc[1]), add2(acc[2], acc[3])), s0, s1);
-      l = l * alpha + (s0 + s1);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(kBarPFull + t));
+      if (!ok) break;
+      // Epilogue: O / l -> bf16 -> global (rows past q_len are not stored).
+      // PV_t of this item's last tile is the (s_it - 1)-th PV of this tile.
+      if (n > 0) {
+        ok = __all_sync(0xffffffffu, wait(kBarODone + t, (s_it - 1) & 1));
+        if (!ok) break;
+        tc_fence_after();
+      }
+      const bool store = row < p.q_len;
+      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.O) +
+                           (((size_t)g.b * p.H + g.h) * p.q_len + (store ? row : 0)) * D;
+      const float inv = (n > 0 && l > 0.f) ? 1.f / l : 0.f;
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t o[32];
+        if (n > 0) {
+          tmem_ld32(tO + 32 * ch, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0u;
+        }
+        if (store) {
+          uint4 packed[4];
+          uint32_t* pw = reinterpret_cast<uint32_t*>(packed);
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pw[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+          uint4* dst = reinterpret_cast<uint4*>(out + 32 * ch);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = packed[i];
+        }
+      }
+      kv_it += g.nmax;
     }
-    if (ok && n > 0) ok = wait(kBarODone + t, (n - 1) & 1);
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok) tc_fence_after();
-    // Epilogue: O / l -> bf16 -> global (rows past q_len are not stored).
-    const bool have_o = ok && n > 0;                 // warp-uniform
-    const bool store = row < g.q_len;
-    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.O) +
-                         (((size_t)g.b * p.H + g.h) * p.q_len + (store ? row : 0)) * D;
-    const float inv = (have_o && l > 0.f) ? 1.f / l : 0.f;
-#pragma unroll
-    for (int ch = 0; ch < 4; ++ch) {
-      uint32_t o[32];
-      if (have_o) {
-        tmem_ld32(tO + 32 * ch, o);
-        tmem_wait_ld();
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] = 0u;
-      }
-      if (store) {
-        uint4 packed[4];
-        uint32_t* pw = reinterpret_cast<uint32_t*>(packed);
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pw[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-        uint4* dst = reinterpret_cast<uint4*>(out + 32 * ch);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) dst[i] = packed[i];
-      }
-    }
+    // No tensor-memory access of this warp may still be in flight at dealloc.
+    tmem_wait_ld();
+    tmem_wait_st();
   }
 
   tc_fence_before();
@@ -643,20 +821,26 @@ bool encode_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint6
          CUDA_SUCCESS;
 }
 
+// Dynamic shared memory is a per-device function attribute; host threads may
+// launch concurrently, so the once-per-device record is kept under a lock.
 template <bool kPaged, bool kFp8QK>
 cudaError_t set_smem_attr() {
-  static int done[64] = {};
+  static bool done[64] = {};
+  static std::mutex mu;
   int dev = 0;
-  cudaGetDevice(&dev);
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
   if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
-  // The in-kernel register split assumes this exact launch allocation.
+  // The in-kernel register split assumes this exact launch allocation (the
+  // build checks it too).
   cudaFuncAttributes fa;
-  cudaError_t e = cudaFuncGetAttributes(&fa, prefill_kernel<kPaged, kFp8QK>);
+  e = cudaFuncGetAttributes(&fa, prefill_kernel<kPaged, kFp8QK>);
   if (e != cudaSuccess) return e;
   if (fa.numRegs != kLaunchRegs) return cudaErrorNotSupported;
   e = cudaFuncSetAttribute(prefill_kernel<kPaged, kFp8QK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kSmemBytes);
-  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = 1;
+  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
   return e;
 }
 
@@ -685,6 +869,8 @@ cudaError_t launch_prefill_bf16(const PrefillParams& p, cudaStream_t stream) {
         !encode_3d(&tv, p.V, D, p.kv_len, bhkv, row_bytes, row_bytes * p.kv_len, BN, 1))
       return cudaErrorInvalidValue;
   }
+  // One CTA per work item; running CTAs claim the items of CTAs that have not
+  // started (so at most one CTA per SM ever runs, and the rest never launch).
   const long long m_blocks = (p.q_len + BM * kQTiles - 1) / (BM * kQTiles);
   const long long ctas = m_blocks * p.B * p.H;
   if (ctas > 0x7fffffffLL) return cudaErrorNotSupported;

@@ -59,6 +59,47 @@ PKV_DEVINLINE bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t lim
   }
 }
 
+// Bounded wait that also gives up as soon as *abort is set (another role of
+// the CTA already gave up): true when the phase completed.
+PKV_DEVINLINE bool mbar_wait_abortable(uint32_t bar, uint32_t parity, uint64_t limit_ns,
+                                       const volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// ------------------------------------------------------ cluster launch control --
+// Ask the hardware to cancel the launch of one CTA of this grid that has not
+// started yet; the 16-byte response lands in shared memory at `resp` and
+// completes 16 bytes of transaction on `bar`.  After a failed request no
+// further request may be made.
+PKV_DEVINLINE void clc_try_cancel(uint32_t resp, uint32_t bar) {
+  asm volatile(
+      "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128"
+      " [%0], [%1];" ::"r"(resp), "r"(bar)
+      : "memory");
+}
+// Decode a response: the cancelled CTA's blockIdx.x, or -1 if none was cancelled.
+PKV_DEVINLINE int clc_cancelled_x(uint32_t resp) {
+  uint32_t ok, x;
+  asm volatile(
+      "{\n\t.reg .b128 r;\n\t.reg .pred p;\n\t"
+      "ld.shared.b128 r, [%2];\n\t"
+      "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t"
+      "clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %1, r;\n\t}"
+      : "=r"(ok), "=r"(x)
+      : "r"(resp)
+      : "memory");
+  return ok ? static_cast<int>(x) : -1;
+}
+
 // --------------------------------------------------------------------- TMA --
 PKV_DEVINLINE void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");

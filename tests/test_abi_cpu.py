@@ -113,6 +113,19 @@ def test_attn_prefill_rejects_bad_arguments(args, status):
                         dtype, None) == status
 
 
+@pytest.mark.parametrize("stall,limit_us,d,status", [
+    (-1, 1000, 128, B.PKV_ERR_INVALID_ARG),        # no tile to stall
+    (2, 0, 128, B.PKV_ERR_INVALID_ARG),            # wait limit below 1 us
+    (2, 10 ** 7 + 1, 128, B.PKV_ERR_INVALID_ARG),  # wait limit above 10 s
+    (2, 1000, 64, B.PKV_ERR_UNSUPPORTED),
+])
+def test_stalled_prefill_hook_rejects_bad_arguments(stall, limit_us, d, status):
+    """The failure-path test hook validates like attn_prefill, plus its own
+    two arguments, before anything is launched."""
+    assert B.raw_status("pkv_test_prefill_stalled", FAKE, FAKE, FAKE, FAKE, 1, 1, 256, d, 1,
+                        ctypes.c_float(0.1), stall, limit_us, None) == status
+
+
 def test_no_alloc_decode_rejects_plans_beyond_its_scratch():
     """A plan whose partials exceed PKV_NOALLOC_SCRATCH_BYTES is refused with
     PKV_ERR_WORKSPACE before anything is launched."""

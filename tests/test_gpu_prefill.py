@@ -168,3 +168,62 @@ def test_chunked_prefill_full_size_sampled_rows():
                            set(np.random.default_rng(81).integers(0, 512, 56).tolist())))
     check_close(got[:, :, rows], paged_ref_per_head(w, rows=rows), "chunked prefill")
     _status_ok()
+
+
+def _ref_without_tokens(w, s, drop):
+    """Oracle for sequence s with the tokens in `drop` left out of the keys.
+
+    The dropped tokens lie in the cached prefix (before the q_len new tokens),
+    which every query row sees, so deleting them keeps every other key's
+    causal visibility: the oracle on the shortened sequence is exact."""
+    L = int(w.seq_lens[s])
+    assert max(drop) < L - w.q_len
+    keep = np.array([t for t in range(L) if t not in set(drop)])
+    table = w.block_table[s].numpy()
+    K = oracle.gather_kv(np_of(w.k_pages), table, L, w.page_size)[:, keep]
+    V = oracle.gather_kv(np_of(w.v_pages), table, L, w.page_size)[:, keep]
+    q = oracle.to_f64(np_of(w.q[s]))
+    H, H_kv = w.q.shape[1], w.k_pages.shape[2]
+    return np.stack([oracle.attention_ref(q[h], K[h // (H // H_kv)], V[h // (H // H_kv)],
+                                          True, w.scale) for h in range(H)])
+
+
+@pytest.mark.parametrize("ps,lens,q_len,bad_page", [(16, [400, 517], 100, 3),
+                                                    (256, [700, 900], 200, 1)])
+def test_paged_prefill_bad_page_is_left_out_and_flagged(ps, lens, q_len, bad_page):
+    """A page id outside the pool in sequence 1's table: nothing outside the
+    pool is read, the error is flagged, sequence 0 is untouched, and sequence 1
+    is attention over its other keys (the bad page's keys left out, as the
+    decode kernel does)."""
+    from paged_kv_cache_exact_b200 import binding as B
+    w = make_paged(91 + ps, lens, H=2, d=128, page_size=ps, q_len=q_len, decoys=2)
+    B.pkv_last_device_error()                                  # clear
+    w.block_table[1, bad_page] = w.k_pages.shape[0] + 7        # out of range
+    got = _paged(w)
+    st, bits = B.pkv_last_device_error()
+    assert st == B.PKV_ERR_BAD_TABLE and bits & B.PKV_DEVERR_BAD_PAGE, (st, bits)
+    check_close(got[:1], paged_ref_per_head(w, seqs=[0]), "good sequence")
+    drop = list(range(bad_page * ps, (bad_page + 1) * ps))
+    check_close(got[1], _ref_without_tokens(w, 1, drop), "sequence with a bad page")
+
+
+def test_bounded_wait_runs_out_then_the_next_call_is_correct():
+    """The failure path of the prefill pipeline, without faulting or hanging
+    the GPU: with every wait bounded at 1 ms and one K load never issued, the
+    CTAs waiting for it give up, drain what they issued, free their tensor
+    memory and exit; the device error word says PKV_ERR_TIMEOUT.  The next
+    normal call on the same context is correct against the oracle."""
+    from paged_kv_cache_exact_b200 import api
+    from paged_kv_cache_exact_b200 import binding as B
+    w = make_dense(95, 1, 2, 1024, 128, causal=True)
+    Q, K, V = w.Q.cuda(), w.K.cuda(), w.V.cuda()
+    O = torch.empty_like(Q)
+    B.pkv_last_device_error()                                  # clear
+    B.pkv_test_prefill_stalled(Q, K, V, O, 1, 2, 1024, 128, True, w.scale, 2, 1000)
+    torch.cuda.synchronize()
+    st, bits = B.pkv_last_device_error()
+    assert st == B.PKV_ERR_TIMEOUT and bits & B.PKV_DEVERR_TIMEOUT, (st, bits)
+    got = api.prefill(Q, K, V, True, w.scale).cpu()
+    check_close(got, oracle.mha_ref(f64(w.Q), f64(w.K), f64(w.V), True, w.scale),
+                "prefill after a timed-out call")
+    _status_ok()
