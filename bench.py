@@ -324,6 +324,8 @@ def run_gpu(args, rank, world, dist):
     append = measure_append(device, stream, peaks)
     paged_study = measure_paged_study(dev, stream, peaks)
     fp8 = measure_fp8(dev, stream, peaks)
+    legs = measure_workload_legs(device, stream, peaks,
+                                 cpu=(rank == 0 and world == 1 and not args.no_cpu_baseline))
     total_ms, e2e_ms, pre_ms, dec_ms = reduce_max([total_ms, e2e_ms, pre_ms, dec_ms], dist,
                                                   device)
     ms_step = total_ms / args.steps
@@ -368,6 +370,7 @@ def run_gpu(args, rank, world, dist):
                         "step, pipelined over 2 buffer sets and 3 streams; the KV page pool is "
                         "resident device state"},
         "append": append,
+        "workloads": legs,
         "paged_vs_contiguous": paged_study,
         "fp8_qk_prefill": fp8,
         "gpu_launches": args.steps * meta["launches_per_step"],
@@ -502,6 +505,103 @@ def measure_fp8(dev, stream, peaks, iters=20):
             "ms": ms, "tflops": tf, "frac_of_bf16_peak": tf / peaks["bf16_tflops"]}
 
 
+def _timed_leg(fn, stream, device, min_s=0.4, warmup=3):
+    """Time fn() with CUDA events on `stream` over at least `min_s` seconds of
+    back-to-back calls (after `warmup` untimed ones), sampling the SM clocks
+    over that same region.  Returns (ms per call, calls, clocks)."""
+    import torch
+
+    for _ in range(warmup):
+        fn()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    e0.record(stream)
+    fn()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    iters = max(10, int(min_s * 1e3 / max(e0.elapsed_time(e1), 1e-3)))
+    sampler = ClockSampler(device.index or 0)
+    sampler.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize(device)
+    sampler.mark(True)
+    e0.record(stream)
+    for _ in range(iters):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    sampler.mark(False)
+    clocks = sampler.stop()
+    return e0.elapsed_time(e1) / iters, iters, clocks
+
+
+def gqa_decode_workload():
+    """Grouped-query decode: 64 sequences x 64 query heads over 8 kv heads,
+    d=128 bf16, seq_lens U[512, 8192], 16-token pages (the pages' Llama-3.1-70B
+    head grouping, "Attention Variants: MHA, GQA, MQA", on the paged-decode
+    length mix)."""
+    from paged_kv_cache_exact_b200.workloads import make_paged
+    return make_paged(2003, (512, 8192, 64), 64, 128, 16, q_len=1, H_kv=8, decoys=64)
+
+
+def measure_workload_legs(device, stream, peaks, cpu=True):
+    """The other workloads, each timed alone: paged decode with 256-token
+    pages (16 seqs, seq_lens U[600, 32768], seq 0 = 600 tokens on pages
+    [5, 1, 9]), the 1 x 32 x 32768 paged causal prefill over 128 shuffled pages
+    of 256, and grouped-query decode (64 query heads over 8 kv heads).  Each
+    leg carries its own clocks and, on request, the oracle on a bounded sample
+    of the same inputs."""
+    import torch
+
+    from paged_kv_cache_exact_b200 import accounting, api
+    from paged_kv_cache_exact_b200.workloads import workload
+    legs = {}
+
+    def paged_inputs(w):
+        t = [x.to(device) for x in (w.q, w.k_pages, w.v_pages, w.block_table, w.seq_lens)]
+        out = torch.empty_like(t[0])
+        ws = api.workspace_for(w.num_seqs, w.q.shape[1], 128, w.max_seq_len, w.page_size, device)
+        fn = lambda: api.paged(*t, w.page_size, True, w.scale, max_seq_len=w.max_seq_len,
+                               out=out, workspace=ws, stream=stream)
+        return t, fn
+
+    for name, w, desc in (
+            ("decode_cfg4", workload(4), "paged decode, 16 seqs x 32 heads, d=128 bf16, "
+             "seq_lens U[600,32768], page_size 256, seq 0 = 600 tokens on pages [5,1,9]"),
+            ("decode_gqa", gqa_decode_workload(), "paged decode, 64 seqs x 64 query heads over "
+             "8 kv heads, d=128 bf16, seq_lens U[512,8192], page_size 16")):
+        t, fn = paged_inputs(w)
+        ms, iters, clocks = _timed_leg(fn, stream, device)
+        H, H_kv = w.q.shape[1], w.k_pages.shape[2]
+        nbytes = accounting.decode_bytes(w.seq_lens.tolist(), H, H_kv, 128,
+                                         max_pages=w.block_table.shape[1])
+        gbs = nbytes / (ms / 1e3) / 1e9
+        leg = {"workload": desc, "ms": ms, "calls": iters, "kv_gbs": gbs,
+               "frac": gbs / peaks["hbm_gbs"], "bytes": nbytes,
+               "sum_seq_lens": int(w.seq_lens.sum()), "clocks": clocks,
+               "l2": f"KV pool {t[1].numel() * 4 / 1e9:.2f} GB > L2"}
+        if cpu:
+            leg["cpu_baseline"] = oracle_decode_sample(w)
+        legs[name] = leg
+        del t, fn
+
+    w = workload(5)
+    t, fn = paged_inputs(w)
+    ms, iters, clocks = _timed_leg(fn, stream, device)
+    flops = accounting.prefill_flops(1, 32, 32768, 32768, 128, True)
+    tf = flops / (ms / 1e3) / 1e12
+    tpeak, tsrc = tensor_peak(peaks, ms * iters / 1e3)
+    leg = {"workload": "paged causal prefill 1x32x32768 d=128 bf16, 128 shuffled pages of 256 "
+                       "(pool of 256 pages, the rest NaN-poisoned)",
+           "ms": ms, "calls": iters, "tflops": tf, "frac": tf / peaks["bf16_tflops"],
+           "frac_of_peak_used": tf / tpeak, "peak_source": tsrc, "flops": flops,
+           "clocks": clocks}
+    if cpu:
+        leg["cpu_baseline"] = oracle_long_prefill_sample(w)
+    legs["paged_prefill_cfg5"] = leg
+    return legs
+
+
 def measure_append(device, stream, peaks, iters=50):
     import torch
 
@@ -573,6 +673,66 @@ class OracleSample:
         return flops, dbytes
 
 
+def oracle_decode_sample(w, budget_s=3.0):
+    """The oracle on (sequence, query head) pairs of a decode workload, for
+    about `budget_s` seconds, in the same unit as the GPU leg (GB/s of K/V;
+    with grouped heads each query head counts its share of its kv head's
+    rows, so the bytes of a whole group are counted once)."""
+    import oracle
+    import torch
+    q = w.q.view(torch.int16).numpy()
+    kp, vp = w.k_pages.view(torch.int16).numpy(), w.v_pages.view(torch.int16).numpy()
+    table, lens = w.block_table.numpy(), w.seq_lens.numpy()
+    S, H, H_kv = q.shape[0], q.shape[1], kp.shape[2]
+    group = H // H_kv
+    nbytes = pairs = 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < budget_s and pairs < S * H:
+        s, h = pairs % S, (pairs // S) % H
+        kvh = h // group
+        oracle.paged_attention_ref(q[s:s + 1, h:h + 1], kp[:, :, kvh:kvh + 1],
+                                   vp[:, :, kvh:kvh + 1], table[s:s + 1], lens[s:s + 1],
+                                   w.page_size, True, w.scale)
+        nbytes += int(lens[s]) * 128 * 2 * 2 / group   # this head's share of its kv head's rows
+        pairs += 1
+    dt = time.perf_counter() - t0
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s of K/V", "cores": _blas_threads(),
+            "kind": "oracle", "sample": f"fp64 NumPy oracle on {pairs} (sequence, query head) "
+                                        f"pairs of the same inputs, {dt:.1f} s"}
+
+
+def oracle_long_prefill_sample(w, rows=512):
+    """The oracle on every head of the long paged prefill at `rows` fixed query
+    rows (the parity test's row mix), and a labelled linear extrapolation to
+    all 32768 rows (the oracle forms each sampled row's scores against all
+    keys, so its cost per row does not depend on the row)."""
+    import numpy as np
+
+    import oracle
+    import torch
+    rng = np.random.default_rng(5)
+    fixed = {0, 1, 127, 128, 255, 256, 257, 16383, 32766, 32767}
+    rest = [int(r) for r in rng.permutation(32768) if int(r) not in fixed][:rows - len(fixed)]
+    sel = np.array(sorted(fixed | set(rest)))
+    q = w.q.view(torch.int16).numpy()
+    kp, vp = w.k_pages.view(torch.int16).numpy(), w.v_pages.view(torch.int16).numpy()
+    table, lens = w.block_table.numpy(), w.seq_lens.numpy()
+    t0 = time.perf_counter()
+    for h in range(q.shape[1]):                  # one head at a time: bounded host memory
+        oracle.paged_attention_ref(q[:, h:h + 1], kp[:, :, h:h + 1], vp[:, :, h:h + 1], table,
+                                   lens, w.page_size, True, w.scale, rows=sel)
+    dt = time.perf_counter() - t0
+    flops = 4 * 128 * 32 * int(sum(int(r) + 1 for r in sel))     # visible pairs of the sample
+    full_s = dt * 32768 / len(sel)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s (visible pairs)",
+            "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"fp64 NumPy oracle, all 32 heads x {len(sel)} fixed query rows of the same "
+                      f"inputs, {dt:.1f} s",
+            "extrapolated_full_s": full_s,
+            "extrapolation": f"linear in rows: {dt:.1f} s x 32768 / {len(sel)} = {full_s:.0f} s "
+                             "for the whole prefill (label: extrapolated, not run)"}
+
+
 def cpu_baseline(peaks, budget_s=12.0, pre=None, dec=None):
     """The oracle as it stands, on rank 0's host cores, for about `budget_s`."""
     smp = OracleSample(pre, dec)
@@ -636,6 +796,8 @@ PROFILE_CASES = {
     "append": "paged KV append, 64 seqs x 512 new tokens, H_kv=32 d=128 bf16, page 16",
     "decode-gqa": "paged decode with grouped heads, 64 seqs x 64 query heads over 8 kv heads, "
                   "seq_lens U[512,8192], page_size 16",
+    "decode256": "paged decode, 16 seqs x 32 heads, seq_lens U[600,32768], page_size 256, "
+                 "seq 0 = 600 tokens on pages [5,1,9]",
 }
 
 
@@ -672,8 +834,10 @@ def run_profile(args):
     else:
         if args.profile == "paged-prefill":
             w = workload(5)
+        elif args.profile == "decode256":
+            w = workload(4)
         elif args.profile == "decode-gqa":
-            w = make_paged(2003, (512, 8192, 64), 64, 128, 16, q_len=1, H_kv=8, decoys=64)
+            w = gqa_decode_workload()
         else:
             w = make_paged(1003, (512, 8192, 16), 32, 128, 16, q_len=1, decoys=16)
         t = [x.to(dev) for x in (w.q, w.k_pages, w.v_pages, w.block_table, w.seq_lens)]
@@ -685,7 +849,7 @@ def run_profile(args):
         fn()
     torch.cuda.synchronize(dev)
     units = (int(w.seq_lens.sum()) * w.k_pages.shape[2]
-             if args.profile in ("decode16", "decode-gqa") else None)
+             if args.profile in ("decode16", "decode-gqa", "decode256") else None)
     print(json.dumps({"profile": args.profile, "case": PROFILE_CASES[args.profile],
                       "iterations": args.steps, "decode_units": units}))
 

@@ -179,7 +179,8 @@ def _ref_without_tokens(w, s, drop):
     L = int(w.seq_lens[s])
     assert max(drop) < L - w.q_len
     keep = np.array([t for t in range(L) if t not in set(drop)])
-    table = w.block_table[s].numpy()
+    table = w.block_table[s].numpy().copy()
+    table[table >= w.k_pages.shape[0]] = 0        # any page: its tokens are dropped below
     K = oracle.gather_kv(np_of(w.k_pages), table, L, w.page_size)[:, keep]
     V = oracle.gather_kv(np_of(w.v_pages), table, L, w.page_size)[:, keep]
     q = oracle.to_f64(np_of(w.q[s]))
