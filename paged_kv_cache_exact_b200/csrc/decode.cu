@@ -262,14 +262,12 @@ constexpr int kGqaThreads = kGqaWarps * 32;
 constexpr int kChunk = 16;                          // tokens per warp step
 constexpr int kRowBytes = D * 2;                    // 256 B per token row
 constexpr int kStageBytes = kChunk * kRowBytes;     // 4 KB per matrix per stage
-#ifndef PKV_GQA_STAGES
-#define PKV_GQA_STAGES 2
-#endif
-constexpr int kGqaStages = PKV_GQA_STAGES;          // cp.async ring depth per warp
-#ifndef PKV_GQA_CTAS_PER_SM
-#define PKV_GQA_CTAS_PER_SM 8
-#endif
-constexpr int kGqaCtasPerSm = PKV_GQA_CTAS_PER_SM;  // split planning target
+// Ring depth per warp and the split-planning target: 2 stages keep shared
+// memory at 65 KB per CTA (3 CTAs = 12 warps per SM), which measured faster
+// than 3 stages at 2 CTAs per SM; finer splits (more CTAs per SM) measured
+// slower.
+constexpr int kGqaStages = 2;                        // cp.async ring depth per warp
+constexpr int kGqaCtasPerSm = 8;                     // split planning target
 constexpr int kWarpSmem = kGqaStages * 2 * kStageBytes;   // stages x (K, V)
 
 PKV_DEVINLINE void cp_async16(uint32_t dst, const void* src, bool valid) {
@@ -279,7 +277,6 @@ PKV_DEVINLINE void cp_async16(uint32_t dst, const void* src, bool valid) {
 }
 PKV_DEVINLINE void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 PKV_DEVINLINE void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-PKV_DEVINLINE void cp_async_wait_2() { asm volatile("cp.async.wait_group 2;" ::: "memory"); }
 PKV_DEVINLINE void cp_async_wait_0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 PKV_DEVINLINE void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
@@ -406,30 +403,36 @@ decode_gqa_kernel(const DecodeParams p) {
     const int ahead = c + (kGqaStages - 1) * kGqaWarps;
     if (ahead < n_chunks) prefetch(ahead, (st + kGqaStages - 1) % kGqaStages);
     cp_async_commit();
-    if (kGqaStages == 3)                             // this chunk's group is complete
-      cp_async_wait_2();
-    else
-      cp_async_wait_1();
+    cp_async_wait_1();                               // this chunk's group is complete
     __syncwarp();
 
-    // S = Q K^T for 16 tokens: two n-tiles of 8 tokens
+    // S = Q K^T for 16 tokens: two n-tiles of 8 tokens, each accumulated in
+    // two halves of the head dimension (two independent MMA chains)
     float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    float sd[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
       const int mi = lane >> 3, ri = lane & 7;
       uint32_t b[4];
       ldsm_x4(k_stage(st) + swz(8 * (mi >> 1) + ri, 2 * kk + (mi & 1)), b);
-      mma_bf16_16816(sc[0], qa[kk], b[0], b[1]);
-      mma_bf16_16816(sc[1], qa[kk], b[2], b[3]);
+      mma_bf16_16816(kk & 1 ? sd[0] : sc[0], qa[kk], b[0], b[1]);
+      mma_bf16_16816(kk & 1 ? sd[1] : sc[1], qa[kk], b[2], b[3]);
     }
-    // online softmax per query head (rows g and g + 8), base 2
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sc[nt][e] += sd[nt][e];
+    // online softmax per query head (rows g and g + 8), base 2.  A chunk lies
+    // in one page (pages hold >= 16 tokens, chunks start 16-aligned); keys of
+    // a page outside the pool are left out.
     const int tok0 = t_begin + c * kChunk;
+    const bool page_ok = s_pages[(tok0 >> p.page_shift) - lp0] >= 0;
     float mx_lo = -INFINITY, mx_hi = -INFINITY;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const bool valid = tok0 + 8 * nt + 2 * t4 + e < t_end;
+        const bool valid = page_ok && tok0 + 8 * nt + 2 * t4 + e < t_end;
         sc[nt][e] = valid ? sc[nt][e] * p.scale_log2 : -INFINITY;
         sc[nt][2 + e] = valid ? sc[nt][2 + e] * p.scale_log2 : -INFINITY;
         mx_lo = fmaxf(mx_lo, sc[nt][e]);
@@ -439,10 +442,16 @@ decode_gqa_kernel(const DecodeParams p) {
     mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 2));
     mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 1));
     mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 2));
-    const float mn_lo = fmaxf(m_lo, mx_lo), mn_hi = fmaxf(m_hi, mx_hi);
-    const float a_lo = ex2(m_lo - mn_lo), a_hi = ex2(m_hi - mn_hi);   // -inf - x -> 0
+    // Reference max per query head, moved only when the chunk's max exceeds
+    // it by more than 2^8 (exact: O and l share it; p stays <= 2^8).
+    const float mn_lo = mx_lo > m_lo + 8.f || (m_lo == -INFINITY && mx_lo != -INFINITY) ? mx_lo : m_lo;
+    const float mn_hi = mx_hi > m_hi + 8.f || (m_hi == -INFINITY && mx_hi != -INFINITY) ? mx_hi : m_hi;
+    // rescale factors: 1 when the reference stays (also -inf, no key yet), 0 from -inf
+    const float a_lo = mn_lo == m_lo ? 1.f : ex2(m_lo - mn_lo);
+    const float a_hi = mn_hi == m_hi ? 1.f : ex2(m_hi - mn_hi);
     const float sub_lo = mn_lo == -INFINITY ? 0.f : mn_lo;
     const float sub_hi = mn_hi == -INFINITY ? 0.f : mn_hi;
+    const bool moved = __any_sync(0xffffffffu, mn_lo != m_lo || mn_hi != m_hi);
     m_lo = mn_lo;
     m_hi = mn_hi;
     float pr[2][4];
@@ -455,12 +464,14 @@ decode_gqa_kernel(const DecodeParams p) {
       }
     l_lo = l_lo * a_lo + (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
     l_hi = l_hi * a_hi + (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]);
+    if (moved) {                                     // warp-uniform
 #pragma unroll
-    for (int i = 0; i < D / 8; ++i) {
-      o[i][0] *= a_lo;
-      o[i][1] *= a_lo;
-      o[i][2] *= a_hi;
-      o[i][3] *= a_hi;
+      for (int i = 0; i < D / 8; ++i) {
+        o[i][0] *= a_lo;
+        o[i][1] *= a_lo;
+        o[i][2] *= a_hi;
+        o[i][3] *= a_hi;
+      }
     }
     // P as the A operand: k = the chunk's 16 tokens
     uint32_t pa[4];

@@ -6,7 +6,7 @@ import torch
 
 import oracle
 from paged_kv_cache_exact_b200.workloads import make_paged, workload
-from tests._util import check_close, paged_ref_per_head, to_dev
+from tests._util import check_close, np_of, paged_ref_per_head, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -132,6 +132,34 @@ def test_bad_page_id_is_flagged_not_faulted():
     assert st == B.PKV_ERR_BAD_TABLE and bits & B.PKV_DEVERR_BAD_PAGE
     # sequence 0 is untouched by the bad entry
     check_close(got[:1], paged_ref_per_head(w, seqs=[0]), "good sequence")
+
+
+@pytest.mark.parametrize("ps,bad_page", [(16, 0), (16, 5), (256, 1)])
+def test_grouped_decode_bad_page_is_left_out_and_flagged(ps, bad_page):
+    """Grouped heads (8 query heads over 2 kv heads) with a page id outside the
+    pool in sequence 1's table: flagged, sequence 0 untouched, and sequence 1
+    is attention over its other tokens (decode sees every token, so leaving
+    the page's tokens out equals the oracle on the shortened sequence).  Page
+    0 is every split's first page of that sequence, so a warp starts on it."""
+    from paged_kv_cache_exact_b200 import binding as B
+    w = make_paged(18 + ps, [700, 1500], H=8, H_kv=2, d=128, page_size=ps, q_len=1)
+    _device_status()                                       # clear
+    w.block_table[1, bad_page] = w.k_pages.shape[0] + 3
+    got = _run(w)
+    st, bits = _device_status()
+    assert st == B.PKV_ERR_BAD_TABLE and bits & B.PKV_DEVERR_BAD_PAGE
+    check_close(got[:1], paged_ref_per_head(w, seqs=[0]), "good sequence")
+    L = int(w.seq_lens[1])
+    drop = set(range(bad_page * ps, (bad_page + 1) * ps))
+    keep = np.array([t for t in range(L) if t not in drop])
+    table = w.block_table[1].numpy().copy()
+    table[table >= w.k_pages.shape[0]] = 0                 # any page: its tokens are dropped
+    K = oracle.gather_kv(np_of(w.k_pages), table, L, ps)[:, keep]
+    V = oracle.gather_kv(np_of(w.v_pages), table, L, ps)[:, keep]
+    q = oracle.to_f64(np_of(w.q[1]))
+    want = np.stack([oracle.attention_ref(q[h], K[h // 4], V[h // 4], True, w.scale)
+                     for h in range(8)])
+    check_close(got[1], want, "sequence with a bad page")
 
 
 @pytest.mark.parametrize("H,H_kv", [(8, 4), (16, 4), (32, 4), (16, 1), (64, 2)])

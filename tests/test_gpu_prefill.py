@@ -61,13 +61,17 @@ def test_dense_large_scores_no_overflow():
     check_close(got, want, "dense large scores")
 
 
-@pytest.mark.parametrize("growth", [7.5, 12.0, 40.0])
+@pytest.mark.parametrize("growth", [7.5, 12.0, 40.0, 100.0])
 @pytest.mark.parametrize("causal", [True, False])
 def test_running_max_staircase(growth, causal):
-    """Key scores that climb by `growth` (log2 units) per 128-key tile.  At 12
-    and 40 every tile moves the row max more than 8 past the reference max, so
-    O is rescaled at every tile; at 7.5 that happens every second tile, and in
-    between exponentials of up to ~2^7.5 go into P without a rescale."""
+    """Key scores that climb by `growth` (log2 units) per 128-key tile, so each
+    tile's second half holds its largest scores.  The kernel's exponentials use
+    a reference max that moves only when a half tile's row sum passes 2^32:
+    at 7.5 it never moves after the first tile (P reaches ~2^30); at 12 the
+    second half of about every third tile overflows and is redone after O is
+    rescaled with PV's first half already in it; at 40 that happens at every
+    tile; at 100 a tile's first half already overflows (redone before any of
+    P is handed over)."""
     N, d, scale = 1000, 128, 0.088
     g = torch.Generator().manual_seed(77)
     log2e = 1.4426950408889634
