@@ -43,7 +43,7 @@ WORKLOAD = ("serving step: causal prefill B=4 H=32 N=4096 d=128 bf16 + paged dec
             "32 heads d=128 bf16, seq_lens U[512,8192], page_size 16")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-PREFILL_SRC = ["prefill_sm100.cu", "sm100_ptx.cuh", "exp2_poly.cuh", "common.cuh"]
+PREFILL_SRC = ["prefill_sm100.cu", "sm100_ptx.cuh", "common.cuh"]
 DECODE_SRC = ["decode.cu", "common.cuh"]
 
 
@@ -787,6 +787,8 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 
 PROFILE_CASES = {
+    "step": "the serving step: causal prefill B=4 H=32 N=4096 d=128 + paged decode 64 seqs x 32 "
+            "heads, seq_lens U[512,8192], page_size 16 (the bench's timed step, 3 launches/iter)",
     "prefill": "causal prefill B=4 H=32 N=4096 d=128 (the step's prefill, 1 launch/iter)",
     "prefill-fp8": "causal prefill B=4 H=32 N=4096 d=128, e4m3 Q/K with per-tensor scales, "
                    "bf16 V/O",
@@ -807,6 +809,18 @@ def run_profile(args):
     from paged_kv_cache_exact_b200 import api
     from paged_kv_cache_exact_b200.workloads import make_paged, workload
     dev = torch.device("cuda", 0)
+    if args.profile == "step":
+        torch.cuda.set_device(dev)
+        prefill, decode, _, _, meta = build_step(dev)
+        stream = torch.cuda.current_stream(dev)
+        for _ in range(args.steps):
+            prefill(stream)
+            decode(stream)
+        torch.cuda.synchronize(dev)
+        print(json.dumps({"profile": "step", "case": PROFILE_CASES["step"],
+                          "iterations": args.steps,
+                          "launches_per_step": meta["launches_per_step"]}))
+        return
     if args.profile == "append":
         run, moved, desc = append_setup(dev)
         for _ in range(args.steps):

@@ -21,7 +21,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libpkv.so")
 SOURCES = ["pkv_api.cu", "decode.cu", "decode_noalloc.cu", "simt_fp32.cu", "prefill_sm100.cu",
            "kv_write.cu", "allocator.cpp"]
-HEADERS = ["common.cuh", "sm100_ptx.cuh", "exp2_poly.cuh"]
+HEADERS = ["common.cuh", "sm100_ptx.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
