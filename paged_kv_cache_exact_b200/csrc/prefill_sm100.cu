@@ -140,7 +140,7 @@ struct Geometry {
 // Work item `item` of the launch order: groups of p.head_group (batch, head)
 // pairs; within a group the heaviest causal Q block of every head comes
 // first, then the next heaviest, ...  The host sizes a group so that its K/V
-// (about 32 MB) stays in L2 while its Q blocks run.
+// (about 64 MB) stays in L2 while its Q blocks run.
 __device__ __forceinline__ Geometry item_geometry(const PrefillParams& p, int item) {
   Geometry g;
   const int m_blocks = (p.q_len + BM * kQTiles - 1) / (BM * kQTiles);
