@@ -64,14 +64,14 @@ def test_dense_large_scores_no_overflow():
 @pytest.mark.parametrize("growth", [7.5, 12.0, 40.0, 100.0])
 @pytest.mark.parametrize("causal", [True, False])
 def test_running_max_staircase(growth, causal):
-    """Key scores that climb by `growth` (log2 units) per 128-key tile, so each
-    tile's second half holds its largest scores.  The kernel's exponentials use
-    a reference max that moves only when a half tile's row sum passes 2^32:
-    at 7.5 it never moves after the first tile (P reaches ~2^30); at 12 the
-    second half of about every third tile overflows and is redone after O is
-    rescaled with PV's first half already in it; at 40 that happens at every
-    tile; at 100 a tile's first half already overflows (redone before any of
-    P is handed over)."""
+    """Key scores that climb by `growth` (log2 units) per 128-key tile, rising
+    key by key, so every row's running max grows at every tile.  The kernel
+    keeps a reference max per row and moves it only when a tile's max passes
+    it by more than 8 (log2 units), rescaling O before any of that tile's P is
+    handed to the PV product: at 7.5 the reference moves every second tile and
+    P reaches about 2^7.5 in the tile between; at 12, 40 and 100 it moves at
+    every tile, and at 100 the rescale factor 2^-100 leaves the earlier O and
+    row sum negligible, as they are in the exact result."""
     N, d, scale = 1000, 128, 0.088
     g = torch.Generator().manual_seed(77)
     log2e = 1.4426950408889634
