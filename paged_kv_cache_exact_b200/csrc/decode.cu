@@ -43,6 +43,7 @@ constexpr int kMaxSplits = 1024;        // splits merged per (sequence, head)
 template <int U>
 __global__ void __launch_bounds__(kThreads)
 decode_split_kernel(const DecodeParams p) {
+  asm volatile("griddepcontrol.launch_dependents;");   // the combine may be scheduled
   const int split = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
   const int tid = threadIdx.x;
 
@@ -191,55 +192,48 @@ decode_split_kernel(const DecodeParams p) {
   }
 }
 
-// Log-sum-exp merge of the splits of one (sequence, head).
-__global__ void __launch_bounds__(D) combine_kernel(const DecodeParams p) {
-  const int h = blockIdx.x, s = blockIdx.y, tid = threadIdx.x;
-  int L = p.seq_lens[s];
+// Log-sum-exp merge of the splits of one (sequence, head), one warp each:
+// lane i owns head dims 4i .. 4i+3 (one 16-byte load per split).  Launched as
+// a programmatic dependent of the split kernel: the grid may be scheduled
+// while the split kernel drains, and waits here until all of its partials are
+// written and visible.
+constexpr int kCombineWarps = 8;
+__global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const DecodeParams p) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const long long sh = (long long)blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (sh >= (long long)p.num_seqs * p.H) return;
+  int L = p.seq_lens[sh / p.H];
   const int cap = min(p.max_seq_len, p.max_pages * p.page_size);
   L = max(0, min(L, cap));
   const int nsplit = (L + p.split_tokens - 1) / p.split_tokens;
   if (nsplit <= 1) return;                          // written by the split kernel
-  const size_t sh = (size_t)s * p.H + h;
   const float2* ml = p.ws_ml + sh * p.max_splits;
-  __shared__ float s_w[kMaxSplits];
-  __shared__ float s_red[D / 32];
-  __shared__ float s_M, s_L;
-  // max over splits
   float M = -INFINITY;
-  for (int j = tid; j < nsplit; j += D) M = fmaxf(M, ml[j].x);
+  for (int j = lane; j < nsplit; j += 32) M = fmaxf(M, ml[j].x);
 #pragma unroll
   for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  if ((tid & 31) == 0) s_red[tid >> 5] = M;
-  __syncthreads();
-  if (tid == 0) {
-    float mm = s_red[0];
-    for (int i = 1; i < D / 32; ++i) mm = fmaxf(mm, s_red[i]);
-    s_M = mm;
-  }
-  __syncthreads();
-  M = s_M;
   float lsum = 0.f;
-  for (int j = tid; j < nsplit; j += D) {
+  for (int j = lane; j < nsplit; j += 32) {
     const float2 v = ml[j];
-    const float w = (M == -INFINITY) ? 0.f : ex2(v.x - M);
-    s_w[j] = w;
-    lsum = fmaf(w, v.y, lsum);
+    lsum = fmaf(M == -INFINITY ? 0.f : ex2(v.x - M), v.y, lsum);
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-  __syncthreads();
-  if ((tid & 31) == 0) s_red[tid >> 5] = lsum;
-  __syncthreads();
-  if (tid == 0) {
-    float t = 0.f;
-    for (int i = 0; i < D / 32; ++i) t += s_red[i];
-    s_L = t;
+  const float4* po = reinterpret_cast<const float4*>(p.ws_o + sh * p.max_splits * D) + lane;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j = 0; j < nsplit; ++j) {
+    const float w = M == -INFINITY ? 0.f : ex2(ml[j].x - M);
+    const float4 x = po[(size_t)j * (D / 4)];
+    acc.x = fmaf(w, x.x, acc.x);
+    acc.y = fmaf(w, x.y, acc.y);
+    acc.z = fmaf(w, x.z, acc.z);
+    acc.w = fmaf(w, x.w, acc.w);
   }
-  __syncthreads();
-  const float* po = p.ws_o + sh * p.max_splits * D + tid;
-  float o = 0.f;
-  for (int j = 0; j < nsplit; ++j) o = fmaf(s_w[j], po[(size_t)j * D], o);
-  p.out[sh * D + tid] = __float2bfloat16_rn(s_L > 0.f ? o / s_L : 0.f);
+  const bool pos = lsum > 0.f;
+  __nv_bfloat162* out = reinterpret_cast<__nv_bfloat162*>(p.out + sh * D) + 2 * lane;
+  out[0] = __floats2bfloat162_rn(pos ? acc.x / lsum : 0.f, pos ? acc.y / lsum : 0.f);
+  out[1] = __floats2bfloat162_rn(pos ? acc.z / lsum : 0.f, pos ? acc.w / lsum : 0.f);
 }
 
 
@@ -305,6 +299,7 @@ PKV_DEVINLINE uint32_t swz(int r, int c) { return r * kRowBytes + ((c ^ (r & 7))
 __global__ void __launch_bounds__(kGqaThreads)
 decode_gqa_kernel(const DecodeParams p) {
   extern __shared__ __align__(128) uint8_t gsm[];
+  asm volatile("griddepcontrol.launch_dependents;");   // the combine may be scheduled
   const int split = blockIdx.x, s = blockIdx.z;
   const int group = p.H / p.H_kv;                    // query heads per kv head
   const int n_hg = (group + 15) / 16;                // 16-head groups per kv head
@@ -557,6 +552,21 @@ void decode_plan(int num_seqs, int H, int max_seq_len, int page_size,
   *max_splits = (max_seq_len + st - 1) / st;
 }
 
+// The combine as a programmatic dependent launch of the split kernel just
+// enqueued on `stream` (it waits for that kernel's results itself).
+static cudaError_t launch_combine(const DecodeParams& q, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(((long long)q.num_seqs * q.H + kCombineWarps - 1) / kCombineWarps));
+  cfg.blockDim = dim3(kCombineWarps * 32);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, combine_kernel, q);
+}
+
 cudaError_t launch_decode_bf16(const DecodeParams& p, cudaStream_t stream) {
   cudaError_t e;
   if (p.H > p.H_kv) {
@@ -592,22 +602,14 @@ cudaError_t launch_decode_bf16(const DecodeParams& p, cudaStream_t stream) {
     decode_gqa_kernel<<<grid, kGqaThreads, smem, stream>>>(q);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    if (q.max_splits > 1) {
-      combine_kernel<<<dim3(p.H, p.num_seqs), D, 0, stream>>>(q);
-      e = cudaGetLastError();
-    }
-    return e;
+    return q.max_splits > 1 ? launch_combine(q, stream) : cudaSuccess;
   } else {
     dim3 grid(p.max_splits, p.H, p.num_seqs);
     decode_split_kernel<4><<<grid, kThreads, 0, stream>>>(p);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (p.max_splits > 1) {
-    combine_kernel<<<dim3(p.H, p.num_seqs), D, 0, stream>>>(p);
-    e = cudaGetLastError();
-  }
-  return e;
+  return p.max_splits > 1 ? launch_combine(p, stream) : cudaSuccess;
 }
 
 }  // namespace pkv

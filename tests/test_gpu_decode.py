@@ -173,6 +173,19 @@ def test_decode_grouped_heads(H, H_kv, ps):
     assert _device_status()[0] == 0
 
 
+def test_decode_grouped_long_split_boundaries():
+    """Grouped heads with enough (sequence, kv head) pairs that the CTAs take
+    2048-key splits (eight times the per-head plan's 256): lengths on every edge of
+    that plan (one key, a multiple of 2048, one past it, one short of it) and
+    random ones, merged by the combine."""
+    edge = [1, 511, 512, 513, 2047, 2048, 2049, 2560, 4096, 4097, 6143, 9000]
+    lens = edge + torch.randint(1, 9001, (64 - len(edge),),
+                                generator=torch.Generator().manual_seed(5)).tolist()
+    w = make_paged(31, lens, H=16, H_kv=4, d=128, page_size=16, q_len=1, decoys=8)
+    check_close(_run(w), paged_ref_per_head(w), "decode grouped, 2048-key splits")
+    assert _device_status()[0] == 0
+
+
 @pytest.mark.slow
 def test_decode_grouped_full_size():
     """64 sequences x 64 query heads over 8 kv heads (Llama-3-70B-like), lengths
