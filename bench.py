@@ -336,8 +336,8 @@ def run_gpu(args, rank, world, dist):
     dec_gbs = meta["decode_bytes"] / (dec_ms / 1e3) / 1e9
     # A tensor-bound kernel is judged against the burst peak unless the timed
     # region lasted long enough for the power cap to set the clocks.
+    tpeak, tsrc = tensor_peak(peaks, total_ms / 1e3, peak_src)
     if pre_ms >= dec_ms:
-        tpeak, tsrc = tensor_peak(peaks, total_ms / 1e3, peak_src)
         roof = {"kernel": "prefill_kernel", "bound": "tensor", "achieved": pre_tf,
                 "peak": tpeak, "unit": "TFLOP/s", "frac": pre_tf / tpeak,
                 "frac_of_burst_peak": pre_tf / peaks["bf16_tflops"],
@@ -361,7 +361,8 @@ def run_gpu(args, rank, world, dist):
                    "l2": "inputs larger than L2 (403 MB prefill Q/K/V, "
                          f"{meta['pool_bytes'] / 1e9:.1f} GB KV pool per step)"},
         "prefill": {"ms": pre_ms, "tflops": pre_tf, "frac": pre_tf / peaks["bf16_tflops"],
-                    "frac_sustained": pre_tf / peaks["bf16_tflops_sustained"]},
+                    "frac_sustained": pre_tf / peaks["bf16_tflops_sustained"],
+                    "frac_of_peak_used": pre_tf / tpeak, "peak_source": tsrc},
         "decode": {"ms": dec_ms, "kv_gbs": dec_gbs, "frac": dec_gbs / peaks["hbm_gbs"]},
         "roofline": roof,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": meta["h2d"],
