@@ -190,6 +190,12 @@ PKV_API size_t paged_attn_workspace_size(int num_seqs, int H, int d, int max_seq
  *               size is 0).  Its contents need no initialisation and are
  *               garbage afterwards.  Two calls in flight at once need two
  *               workspaces.
+ *
+ * Launches (all on `stream`): q_len == 1 enqueues the split kernel and, when
+ * some sequence spans more than one split, a merge kernel after it.  With
+ * H > H_kv the merge is a programmatic dependent launch: it may be scheduled
+ * while the split kernel drains, and it waits on the device for that kernel's
+ * results, so stream order is kept (also under stream capture).
  */
 PKV_API int paged_attn(const void* q, const void* k_pages, const void* v_pages,
                const int32_t* block_table, const int32_t* seq_lens,

@@ -194,3 +194,35 @@ def test_decode_grouped_full_size():
     err, rel = check_close(_run(w), paged_ref_per_head(w), "decode gqa 64/8 full size")
     assert _device_status()[0] == 0
     print(f"gqa 64/8: max abs err {err:.3e}, max rel err {rel:.3e}")
+
+
+@pytest.mark.parametrize("H,H_kv", [(8, 8), (16, 2)])
+def test_decode_captured_in_a_cuda_graph_matches_direct_calls(H, H_kv):
+    """Decode captured into a CUDA graph and replayed gives the direct call's
+    bits: per-head heads (split kernel, then a plain merge launch) and grouped
+    heads (split kernel, then the merge as a programmatic dependent launch),
+    with several splits per sequence so that the merge runs."""
+    from paged_kv_cache_exact_b200 import api
+    w = make_paged(41 + H, [700, 3000, 5000, 1], H=H, H_kv=H_kv, d=128, page_size=16, q_len=1,
+                   decoys=4)
+    d = to_dev(w)
+    ws = api.workspace_for(w.num_seqs, H, 128, w.max_seq_len, 16, d["q"].device)
+    assert ws is not None                                      # several splits per sequence
+    out = torch.empty_like(d["q"])
+
+    def call():
+        api.paged(d["q"], d["k"], d["v"], d["table"], d["lens"], 16, True, w.scale,
+                  max_seq_len=w.max_seq_len, out=out, workspace=ws)
+
+    call()                                                     # first call outside the capture
+    torch.cuda.synchronize()
+    direct = out.clone()
+    out.zero_()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), direct.view(torch.int16))
+    check_close(out.cpu(), paged_ref_per_head(w), f"graph-replayed decode H={H} H_kv={H_kv}")
+    assert _device_status()[0] == 0
