@@ -85,7 +85,7 @@ SUSTAINED_AFTER_S = 1.0
 
 
 def tensor_peak(peaks, timed_s, peak_src="measured"):
-    """The bf16 tensor peak a kernel's TFLOP/s is judged against, and why.
+    """The bf16 tensor peak a kernel's TFLOP/s is measured against, and why.
 
     A kernel timed inside a region of at least SUSTAINED_AFTER_S seconds of
     back-to-back work runs under the 1 kW power cap: the sustained figure
@@ -334,7 +334,7 @@ def run_gpu(args, rank, world, dist):
                                world)
     pre_tf = meta["prefill_flops"] / (pre_ms / 1e3) / 1e12
     dec_gbs = meta["decode_bytes"] / (dec_ms / 1e3) / 1e9
-    # A tensor-bound kernel is judged against the burst peak unless the timed
+    # A tensor-bound kernel is measured against the burst peak unless the timed
     # region lasted long enough for the power cap to set the clocks.
     tpeak, tsrc = tensor_peak(peaks, total_ms / 1e3, peak_src)
     if pre_ms >= dec_ms:
