@@ -31,7 +31,10 @@
  *   (a page id outside [0, num_pages), a sequence length outside its table,
  *   a pipeline wait that ran out) never fault: the kernel skips the access,
  *   records a bit in a library-wide device error word and carries on;
- *   pkv_last_device_error() reads and clears it.
+ *   pkv_last_device_error() reads and clears it.  A page outside the pool is
+ *   never read and its keys are left out of the softmax (decode and prefill
+ *   alike), so that sequence gets attention over its other keys; a length
+ *   outside its table is clamped into range.
  * - Masking: query row i (0-based, of q_len rows) may see key j (of kv_len keys)
  *   iff j <= i + (kv_len - q_len) when causal, every j < kv_len otherwise.
  *   With q_len == kv_len that is the lower triangle; with q_len == 1 (decode)
@@ -77,7 +80,7 @@ typedef enum {
 typedef enum { PKV_F32 = 0, PKV_BF16 = 1 } pkv_dtype;
 
 /* Device error bits, as returned in *bits by pkv_last_device_error(). */
-#define PKV_DEVERR_BAD_PAGE 0x1u   /* block_table entry outside [0, num_pages): page skipped */
+#define PKV_DEVERR_BAD_PAGE 0x1u   /* block_table entry outside [0, num_pages): its keys left out */
 #define PKV_DEVERR_BAD_LEN 0x2u    /* seq_len outside [q_len, min(max_seq_len, pages*page_size)] */
 #define PKV_DEVERR_TIMEOUT 0x4u    /* a bounded mbarrier wait ran out; the tile was abandoned */
 
